@@ -1,0 +1,63 @@
+"""Seeded synthetic inputs for the attention library and its checks.
+
+This module holds no attention arithmetic: it only draws random bf16 tensors.
+It is the one piece of code that both the CUDA path (tests, bench) and the CPU
+oracle's callers use, so that both see the same bits.
+
+Recipe (the FlashAttention-2 kernel benchmark isolates attention on random
+inputs; no dataset is involved):
+  * "normal":     Q, K, V (and dO) i.i.d. N(0, 1) in fp32, rounded to bf16
+                  (round-to-nearest-even, torch's cast).
+  * "row_scaled": each (b, h, n) row of Q, K and V is N(0, 0.5^2) times a
+                  factor r ~ U(0.5, 2) drawn per row and per tensor; dO stays
+                  N(0, 1).  This varies score magnitudes as in GPT-style layers.
+All draws come from one ``torch.Generator('cpu')`` seeded with ``seed``, in the
+order q, k, v, dO, so a given (shape, seed, dist) always yields the same bits.
+"""
+from __future__ import annotations
+
+import math
+import numpy as np
+import torch
+
+
+def _normal(gen: torch.Generator, shape, std: float = 1.0) -> torch.Tensor:
+    x = torch.randn(shape, generator=gen, dtype=torch.float32)
+    if std != 1.0:
+        x = x * std
+    return x
+
+
+def _row_scaled(gen: torch.Generator, shape) -> torch.Tensor:
+    x = _normal(gen, shape, 0.5)
+    r = torch.rand(shape[:-1] + (1,), generator=gen, dtype=torch.float32)
+    return x * (0.5 + 1.5 * r)
+
+
+def attention_inputs(B: int, H: int, N: int, d: int, seed: int,
+                     dist: str = "normal", with_dout: bool = False):
+    """Return a dict of CPU bf16 tensors q, k, v (and dO) of shape [B,H,N,d]."""
+    gen = torch.Generator("cpu").manual_seed(int(seed))
+    shape = (B, H, N, d)
+    out = {}
+    for name in ("q", "k", "v"):
+        if dist == "normal":
+            x = _normal(gen, shape)
+        elif dist == "row_scaled":
+            x = _row_scaled(gen, shape)
+        else:
+            raise ValueError(f"unknown input distribution {dist!r}")
+        out[name] = x.to(torch.bfloat16)
+    if with_dout:
+        out["dO"] = _normal(gen, shape).to(torch.bfloat16)
+    return out
+
+
+def default_scale(d: int) -> float:
+    """1/sqrt(d) rounded to fp32, the value both sides receive."""
+    return float(np.float32(1.0 / math.sqrt(d)))
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    """Widen a bf16/fp32 CPU tensor exactly to a float64 numpy array."""
+    return t.detach().to("cpu", torch.float64).numpy()

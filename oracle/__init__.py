@@ -1,0 +1,178 @@
+"""fp64 CPU oracle for exact attention -- TEST INFRASTRUCTURE ONLY.
+
+The plain definition of scaled-dot-product attention and its gradient, in
+double precision, written in C (``attention_ref.c``) and loaded here with
+ctypes.  Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU
+baseline leg may import this package.  It shares no code with the CUDA library
+and never calls it; the CUDA library never calls it either.
+
+Every function takes float64 numpy arrays in the [B,H,N,d] layout (LSE and D
+are [B,H,N]) and returns float64 arrays.  Bf16 inputs are widened exactly by
+the caller, so the oracle sees the same values the GPU does.
+
+Parity pins: every function here is pinned by ``tests/test_oracle.py`` against
+quantities fixed by mathematics rather than by this code (high-precision brute
+force, numerical derivatives, closed forms, invariants and an independent
+library routine).  No function is "parity unpinned".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attention_ref.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+_D = ctypes.POINTER(ctypes.c_double)
+_LL = ctypes.POINTER(ctypes.c_longlong)
+
+
+def build(src: str = _SRC, out: str = _LIB_PATH) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP, strict IEEE double)."""
+    cmd = ["gcc", "-O2", "-fopenmp", "-fno-fast-math", "-ffp-contract=off",
+           "-shared", "-fPIC", "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+    return out
+
+
+def open_library(path: str):
+    """Load an oracle build from ``path`` and declare its C signatures."""
+    lib = ctypes.CDLL(path)
+    i, d = ctypes.c_int, ctypes.c_double
+    lib.ref_fwd.argtypes = [_D, _D, _D, _D, _D, i, i, i, i, i, d]
+    lib.ref_fwd.restype = i
+    lib.ref_bwd.argtypes = [_D, _D, _D, _D, _D, _D, _D, _D, i, i, i, i, i, d]
+    lib.ref_bwd.restype = i
+    lib.ref_fwd_rows.argtypes = [_D, _D, _D, i, i, i, d, _LL, i, _D, _D]
+    lib.ref_fwd_rows.restype = i
+    lib.ref_head_stats.argtypes = [_D, _D, _D, _D, i, i, i, d, _D, _D]
+    lib.ref_head_stats.restype = i
+    lib.ref_dq_rows.argtypes = [_D, _D, _D, _D, i, i, i, d, _LL, i, _D]
+    lib.ref_dq_rows.restype = i
+    lib.ref_dkdv_rows.argtypes = [_D, _D, _D, _D, _D, _D, i, i, i, d, _LL, i,
+                                  _D, _D]
+    lib.ref_dkdv_rows.restype = None
+    lib.ref_num_threads.argtypes = []
+    lib.ref_num_threads.restype = i
+    return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        if (not os.path.exists(_LIB_PATH)
+                or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC)):
+            build()
+        _lib = open_library(_LIB_PATH)
+    return _lib
+
+
+def _f64(x) -> np.ndarray:
+    a = np.ascontiguousarray(x, dtype=np.float64)
+    return a
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(_D)
+
+
+def num_threads() -> int:
+    return _load().ref_num_threads()
+
+
+def ref_fwd(q, k, v, causal: bool, scale: float, lib=None):
+    """O and LSE of softmax(scale * Q K^T [causal]) V for [B,H,N,d] inputs."""
+    lib = lib or _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    o = np.empty_like(q)
+    lse = np.empty((B, H, N), dtype=np.float64)
+    if N:
+        rc = lib.ref_fwd(_p(q), _p(k), _p(v), _p(o), _p(lse), B, H, N, d,
+                         int(bool(causal)), float(scale))
+        if rc:
+            raise MemoryError("oracle forward: allocation failed")
+    return o, lse
+
+
+def ref_bwd(q, k, v, dO, causal: bool, scale: float, lib=None):
+    """dQ, dK, dV and D = rowsum(P * dP) for upstream gradient dO."""
+    lib = lib or _load()
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    B, H, N, d = q.shape
+    dq, dk, dv = np.empty_like(q), np.empty_like(q), np.empty_like(q)
+    D = np.empty((B, H, N), dtype=np.float64)
+    if N:
+        rc = lib.ref_bwd(_p(q), _p(k), _p(v), _p(dO), _p(dq), _p(dk), _p(dv),
+                         _p(D), B, H, N, d, int(bool(causal)), float(scale))
+        if rc:
+            raise MemoryError("oracle backward: allocation failed")
+    return dq, dk, dv, D
+
+
+def _rows(rows) -> np.ndarray:
+    return np.ascontiguousarray(rows, dtype=np.int64)
+
+
+def ref_fwd_rows(q, k, v, rows, causal: bool, scale: float, lib=None):
+    """O and LSE for the query ``rows`` of one head; q,k,v are [N,d]."""
+    lib = lib or _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    N, d = q.shape
+    r = _rows(rows)
+    o = np.empty((len(r), d), dtype=np.float64)
+    lse = np.empty(len(r), dtype=np.float64)
+    rc = lib.ref_fwd_rows(_p(q), _p(k), _p(v), N, d, int(bool(causal)),
+                          float(scale), r.ctypes.data_as(_LL), len(r), _p(o),
+                          _p(lse))
+    if rc:
+        raise MemoryError("oracle: allocation failed")
+    return o, lse
+
+
+def ref_head_stats(q, k, v, dO, causal: bool, scale: float, lib=None):
+    """LSE_i and D_i for every query row of one head ([N,d] inputs)."""
+    lib = lib or _load()
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    N, d = q.shape
+    lse = np.empty(N, dtype=np.float64)
+    D = np.empty(N, dtype=np.float64)
+    rc = lib.ref_head_stats(_p(q), _p(k), _p(v), _p(dO), N, d,
+                            int(bool(causal)), float(scale), _p(lse), _p(D))
+    if rc:
+        raise MemoryError("oracle: allocation failed")
+    return lse, D
+
+
+def ref_dq_rows(q, k, v, dO, rows, causal: bool, scale: float, lib=None):
+    """dQ for the query ``rows`` of one head."""
+    lib = lib or _load()
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    N, d = q.shape
+    r = _rows(rows)
+    dq = np.empty((len(r), d), dtype=np.float64)
+    rc = lib.ref_dq_rows(_p(q), _p(k), _p(v), _p(dO), N, d, int(bool(causal)),
+                         float(scale), r.ctypes.data_as(_LL), len(r), _p(dq))
+    if rc:
+        raise MemoryError("oracle: allocation failed")
+    return dq
+
+
+def ref_dkdv_rows(q, k, v, dO, lse, D, rows, causal: bool, scale: float,
+                  lib=None):
+    """dK and dV for the key ``rows`` of one head, given all rows' LSE and D."""
+    lib = lib or _load()
+    q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
+    lse, D = _f64(lse), _f64(D)
+    N, d = q.shape
+    r = _rows(rows)
+    dk = np.empty((len(r), d), dtype=np.float64)
+    dv = np.empty((len(r), d), dtype=np.float64)
+    lib.ref_dkdv_rows(_p(q), _p(k), _p(v), _p(dO), _p(lse), _p(D), N, d,
+                      int(bool(causal)), float(scale), r.ctypes.data_as(_LL),
+                      len(r), _p(dk), _p(dv))
+    return dk, dv
