@@ -1,0 +1,484 @@
+#!/usr/bin/env python
+"""Benchmark of exact attention (forward + backward) on B200.
+
+One step = the whole hot path on one batch: fa_fwd, then the three backward
+stages (fa_bwd_preprocess, fa_bwd_main, fa_bwd_dq_convert), through the C ABI.
+Throughput is TFLOP/s by the FlashAttention-2 convention: forward
+4*B*H*N^2*d (halved when causal), backward 2.5x forward.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+
+With N > 1 (launched by torchrun) every rank runs its own independent shard of
+heads (weak scaling, no data-path collective); the time is the max over ranks.
+Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("attention fwd / fwd+bwd TFLOP/s (bf16, d=64/128, causal) and % of B200 "
+          "BF16 peak")
+
+# Points of the 16k-token sweep (width 2048, B = 16384 / N) and the GPT layers.
+WORKLOADS = {
+    "fwd_bwd_sweep_N8192_d128_causal": dict(B=2, H=16, N=8192, d=128, causal=True,
+                                            dist="normal", seed=2),
+    "fwd_bwd_sweep_N16384_d128_causal": dict(B=1, H=16, N=16384, d=128, causal=True,
+                                             dist="normal", seed=2),
+    "fwd_bwd_sweep_N2048_d128_causal": dict(B=8, H=16, N=2048, d=128, causal=True,
+                                            dist="normal", seed=2),
+    "fwd_bwd_sweep_N8192_d64_causal": dict(B=2, H=32, N=8192, d=64, causal=True,
+                                           dist="normal", seed=2),
+    "fwd_bwd_sweep_N8192_d128_noncausal": dict(B=2, H=16, N=8192, d=128, causal=False,
+                                               dist="normal", seed=2),
+    "gpt_layer_a_B8_N2048_H16_d128": dict(B=8, H=16, N=2048, d=128, causal=True,
+                                          dist="row_scaled", seed=4),
+    "gpt_layer_b_B2_N8192_H20_d128": dict(B=2, H=20, N=8192, d=128, causal=True,
+                                          dist="row_scaled", seed=5),
+}
+DEFAULT_WORKLOAD = "fwd_bwd_sweep_N8192_d128_causal"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+DATASHEET_BF16_TFLOPS = 2250.0
+
+
+def fwd_flops(w) -> float:
+    f = 4.0 * w["B"] * w["H"] * w["N"] ** 2 * w["d"]
+    return f * (0.5 if w["causal"] else 1.0)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", 0) or 0),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def kernel_sources_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_attention_109_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources and this workload; otherwise None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        ent = rec[kernel][workload]
+        if ent.get("sources_hash") != kernel_sources_hash():
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------- clocks
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons (read-only)."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        import torch
+        self.proc = None
+        sel = []
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+        except Exception:
+            sel = []
+        self.cmd = ["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}",
+                    "--format=csv,noheader,nounits", "-lms", "100"]
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [l for l in out.splitlines() if l.strip()]
+        return False
+
+    def summary(self):
+        rows = []
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"],
+                    "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown",
+                 "sw_power_cap"]
+        seen = set()
+        for _, _, flags in rows:
+            for n, fl in zip(names, flags):
+                if fl.lower().startswith("active"):
+                    seen.add(n)
+        return {"sm_mhz": statistics.median(r[0] for r in rows),
+                "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(seen), "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle
+
+
+def oracle_sample(w, seconds: float, seed: int = 0):
+    """Time the fp64 oracle on sampled rows of head 0 of the workload.
+
+    Per-row softmax statistics (LSE_i, D_i) of the head are computed once,
+    untimed; each timed pass then produces O, LSE and dQ for R query rows and
+    dK, dV for R key rows, i.e. R/N of the head's outputs, credited R/N of the
+    head's fwd+bwd FLOPs.  R is sized so one pass takes about `seconds`.
+    Returns (run(R) -> seconds, R, cores, flops_per_pass(R)).
+    """
+    import numpy as np
+    import oracle
+    from exact_attention_109_b200.inputs import attention_inputs, default_scale, to_f64
+
+    inp = attention_inputs(1, 1, w["N"], w["d"], w["seed"], w["dist"], with_dout=True)
+    q, k, v, dO = (to_f64(inp[x])[0, 0] for x in ("q", "k", "v", "dO"))
+    scale = default_scale(w["d"])
+    causal = w["causal"]
+    lse, D = oracle.ref_head_stats(q, k, v, dO, causal, scale)
+    rng = np.random.default_rng(seed)
+    N = w["N"]
+    head = dict(w, B=1, H=1)
+    per_head = 3.5 * fwd_flops(head)
+
+    def run(R):
+        rows = np.sort(rng.choice(N, size=R, replace=False))
+        t0 = time.perf_counter()
+        oracle.ref_fwd_rows(q, k, v, rows, causal, scale)
+        oracle.ref_dq_rows(q, k, v, dO, rows, causal, scale)
+        oracle.ref_dkdv_rows(q, k, v, dO, lse, D, rows, causal, scale)
+        return time.perf_counter() - t0
+
+    r0 = min(N, 256)
+    t = run(r0)
+    R = int(min(N, max(8, math.ceil(r0 * seconds / max(t, 1e-6)))))
+    return run, R, oracle.num_threads(), (lambda r: per_head * r / N)
+
+
+def oracle_whole_heads(w, seconds: float):
+    """Time the fp64 oracle's full forward and backward (ref_fwd, ref_bwd) on
+    whole heads of the workload: as many heads as the host has threads (at most
+    B*H), fewer if one head alone already takes `seconds`."""
+    import oracle
+    from exact_attention_109_b200.inputs import attention_inputs, default_scale, to_f64
+
+    cores = oracle.num_threads()
+    heads = max(1, min(w["B"] * w["H"], cores))
+    inp = attention_inputs(1, heads, w["N"], w["d"], w["seed"], w["dist"], with_dout=True)
+    q, k, v, dO = (to_f64(inp[x]) for x in ("q", "k", "v", "dO"))
+    scale = default_scale(w["d"])
+    t0 = time.perf_counter()
+    oracle.ref_fwd(q, k, v, w["causal"], scale)
+    oracle.ref_bwd(q, k, v, dO, w["causal"], scale)
+    t = time.perf_counter() - t0
+    flops = 3.5 * fwd_flops(dict(w, B=1, H=heads))
+    return flops / t / 1e12, t, heads, cores
+
+
+def reference_arm(args, w, wname):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    steps, warmup = args.steps, args.warmup
+    per_step = max(0.05, 150.0 / max(1, steps + warmup))
+    run, R, cores, credit = oracle_sample(w, per_step)
+    for _ in range(warmup):
+        run(R)
+    times = [run(R) for _ in range(steps)]
+    total = sum(times)
+    value = credit(R) * steps / total / 1e12
+    sample = (f"{R} of {w['N']} query rows (O, LSE, dQ) and key rows (dK, dV) of one "
+              f"head per step, credited {R}/{w['N']} of the head's fwd+bwd FLOPs; "
+              f"per-row LSE/D statistics precomputed untimed")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": steps, "warmup": warmup,
+        "ms_per_step": 1e3 * total / steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, wname),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config(w, wname):
+    return {"workload": wname, "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
+            "causal": w["causal"], "inputs": w["dist"], "pass": "fwd+bwd",
+            "global_batch": w["B"], "seq_len": w["N"],
+            "parallelism": "independent head shards per GPU"}
+
+
+# ---------------------------------------------------------------- GPU arm
+
+
+def gpu_arm(args, w, wname):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_109_b200 as fa
+    from exact_attention_109_b200.inputs import attention_inputs, default_scale
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+
+    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+    scale = default_scale(d)
+    host = attention_inputs(B, H, N, d, w["seed"] + rank, w["dist"], with_dout=True)
+    dev = {k_: v_.cuda() for k_, v_ in host.items()}
+    q, k, v, dO = dev["q"], dev["k"], dev["v"], dev["dO"]
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws_bytes = fa.fa_bwd_workspace_size(B, H, N, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+    P = {x: t.data_ptr() for x, t in dict(q=q, k=k, v=v, dO=dO, o=o, lse=lse, dq=dq,
+                                         dk=dk, dv=dv, ws=ws).items()}
+
+    def stage_fwd():
+        return fa.fa_fwd(P["q"], P["k"], P["v"], P["o"], P["lse"], B, H, N, d, causal,
+                         scale, s)
+
+    def stage_pre():
+        return fa.fa_bwd_preprocess(P["o"], P["lse"], P["dO"], B, H, N, d, P["ws"],
+                                    ws_bytes, s)
+
+    def stage_main():
+        return fa.fa_bwd_main(P["q"], P["k"], P["v"], P["dO"], P["dk"], P["dv"], B, H, N,
+                              d, causal, scale, P["ws"], ws_bytes, s)
+
+    def stage_conv():
+        return fa.fa_bwd_dq_convert(P["dq"], B, H, N, d, scale, P["ws"], ws_bytes, s)
+
+    stages = [("fa_fwd_kernel", stage_fwd), ("fa_bwd_pre_kernel", stage_pre),
+              ("fa_bwd_main_kernel", stage_main), ("fa_bwd_dq_convert_kernel", stage_conv)]
+
+    def step(events=None):
+        for i, (_, fn) in enumerate(stages):
+            if events is not None:
+                events[i].record(stream)
+            st = fn()
+            if st != fa.FA_OK:
+                raise fa.FaError(st, "bench step")
+        if events is not None:
+            events[len(stages)].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    status = fa.fa_get_device_error()
+    if status != fa.FA_OK:
+        raise fa.FaError(status, "warm-up")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)]
+           for _ in range(K)]
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)  # let the sampler start before the timed region
+        torch.cuda.synchronize()
+        for i in range(K):
+            step(evs[i])
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    status = fa.fa_get_device_error()
+    if status != fa.FA_OK:
+        raise fa.FaError(status, "timed region")
+
+    elapsed_ms = evs[0][0].elapsed_time(evs[-1][-1])
+    per_stage = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
+                 for j in range(len(stages))]
+    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=q.device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    elapsed_max = float(t.item())
+
+    flops_step = 3.5 * fwd_flops(w)
+    value = flops_step * K * world / (elapsed_max * 1e-3) / 1e12
+
+    # ---- end to end through the public API with pinned host buffers
+    pin = {x: host[x].pin_memory() for x in ("q", "k", "v", "dO")}
+    out_host = {x: torch.empty(t_.shape, dtype=t_.dtype, pin_memory=True)
+                for x, t_ in dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv).items()}
+    h2d = sum(t_.numel() * t_.element_size() for t_ in pin.values())
+    d2h = sum(t_.numel() * t_.element_size() for t_ in out_host.values())
+
+    def e2e_step():
+        for x in ("q", "k", "v", "dO"):
+            dev[x].copy_(pin[x], non_blocking=True)
+        fa.attention_forward(q, k, v, causal, scale, out=o, lse=lse)
+        fa.attention_backward(q, k, v, o, lse, dO, causal, scale, dq=dq, dk=dk, dv=dv,
+                              workspace=ws)
+        for x, t_ in dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv).items():
+            out_host[x].copy_(t_, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    Ke = max(3, min(K, 20))
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=q.device)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = flops_step * Ke * world / (float(te.item()) * 1e-3) / 1e12
+    status = fa.fa_get_device_error()
+    if status != fa.FA_OK:
+        raise fa.FaError(status, "e2e")
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    # ---- roofline of the dominant kernel
+    peaks = load_peaks()
+    names = [n for n, _ in stages]
+    dom = int(np.argmax(per_stage))
+    bh = B * H
+    n_pad = (N + 127) // 128 * 128
+    algo = {
+        "fa_fwd_kernel": ("tensor", fwd_flops(w)),
+        "fa_bwd_main_kernel": ("tensor", 2.5 * fwd_flops(w)),
+        "fa_bwd_pre_kernel": ("hbm", 2 * bh * N * d * 2 + bh * N * 4 + 2 * bh * n_pad * 4
+                              + bh * n_pad * d * 4),
+        "fa_bwd_dq_convert_kernel": ("hbm", bh * N * d * 4 + bh * N * d * 2),
+    }
+    bound, amount = algo[names[dom]]
+    sec = per_stage[dom] * 1e-3
+    if bound == "tensor":
+        achieved = amount / sec / 1e12
+        peak = peaks["bf16_tflops"]
+        unit = "TFLOP/s"
+    else:
+        achieved = amount / sec / 1e9
+        peak = peaks["hbm_gbs"]
+        unit = "GB/s"
+    roofline = {"kernel": names[dom], "bound": bound, "achieved": achieved, "peak": peak,
+                "unit": unit, "frac": achieved / peak,
+                "peak_source": f"{peaks['source']} (burst)",
+                "traffic": recorded_traffic(names[dom], wname)}
+    fwd_t = fwd_flops(w) / (per_stage[0] * 1e-3) / 1e12
+    bwd_ms = sum(per_stage[1:])
+    bwd_t = 2.5 * fwd_flops(w) / (bwd_ms * 1e-3) / 1e12
+
+    # ---- CPU baseline: the oracle on the host cores, bounded sample
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        val, tcpu, heads, cores = oracle_whole_heads(w, 30.0)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": (f"oracle ref_fwd + ref_bwd on {heads} whole heads of the "
+                          f"workload (N={N}, d={d}, causal={causal}), {tcpu:.1f} s")}
+
+    clocks = clk.summary()
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": elapsed_max / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w, wname),
+                       l2=("no flush: per-step working set "
+                           f"{(9 * bh * N * d * 2 + ws_bytes) / 1e6:.0f} MB > 126 MB L2")),
+        "fwd_tflops": fwd_t, "bwd_tflops": bwd_t,
+        "frac_of_peak": value / peaks["bf16_tflops"],
+        "frac_of_datasheet_bf16": value / DATASHEET_BF16_TFLOPS,
+        "kernel_ms": {n: round(t_, 4) for n, t_ in zip(names, per_stage)},
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": len(stages) * K,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return reference_arm(args, w, args.workload)
+    return gpu_arm(args, w, args.workload)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

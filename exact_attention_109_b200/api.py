@@ -1,11 +1,187 @@
-"""placeholder"""
+"""ctypes binding of libfa_sm100.so -- argument marshalling only.
+
+Every function here converts torch tensors (or raw integers) into the pointers
+and sizes of the C ABI in ``include/fa.h`` and calls the entry point of the same
+name.  All arithmetic happens in the CUDA kernels behind that ABI; there is no
+fallback path, and a missing library raises ``FaError`` on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
 FA_OK = 0
 FA_ERR_INVALID_ARG = 1
 FA_ERR_UNSUPPORTED = 2
 FA_ERR_MISALIGNED = 3
 FA_ERR_CUDA = 4
 FA_ERR_TIMEOUT = 5
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libfa_sm100.so"
+_lib = None
+
+
 class FaError(RuntimeError):
-    pass
-library = library_path = fa_fwd = fa_bwd = fa_bwd_workspace_size = None
-fa_get_device_error = fa_strerror = attention_forward = attention_backward = None
+    """A C entry point returned a status other than FA_OK."""
+
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {fa_strerror(status) if _lib else status}")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def library():
+    """Load the CUDA library (raises when it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise FaError(FA_ERR_UNSUPPORTED,
+                      f"{_LIB_NAME} not built (run __graft_entry__.build())")
+    lib = ctypes.CDLL(path)
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp]
+    lib.fa_fwd.restype = i
+    lib.fa_bwd_workspace_size.argtypes = [i, i, i, i]
+    lib.fa_bwd_workspace_size.restype = sz
+    lib.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f,
+                           vp, sz, vp]
+    lib.fa_bwd.restype = i
+    lib.fa_bwd_preprocess.argtypes = [vp, vp, vp, i, i, i, i, vp, sz, vp]
+    lib.fa_bwd_preprocess.restype = i
+    lib.fa_bwd_main.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz, vp]
+    lib.fa_bwd_main.restype = i
+    lib.fa_bwd_dq_convert.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
+    lib.fa_bwd_dq_convert.restype = i
+    lib.fa_get_device_error.argtypes = [vp]
+    lib.fa_get_device_error.restype = i
+    lib.fa_strerror.argtypes = [i]
+    lib.fa_strerror.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def fa_strerror(status: int) -> str:
+    return library().fa_strerror(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != FA_OK:
+        raise FaError(status, where)
+
+
+# ---------------------------------------------------------------- raw entry points
+
+def fa_fwd(q: int, k: int, v: int, o: int, lse: int, B: int, H: int, N: int,
+           d: int, causal: int, scale: float, stream: int = 0) -> int:
+    """Raw C call with device pointers as integers; returns the status."""
+    return library().fa_fwd(q, k, v, o, lse, B, H, N, d, int(causal),
+                            float(scale), stream or None)
+
+
+def fa_bwd(q: int, k: int, v: int, o: int, lse: int, dO: int, dq: int, dk: int,
+           dv: int, B: int, H: int, N: int, d: int, causal: int, scale: float,
+           workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    """Raw C call with device pointers as integers; returns the status."""
+    return library().fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d,
+                            int(causal), float(scale), workspace,
+                            int(workspace_bytes), stream or None)
+
+
+def fa_bwd_preprocess(o: int, lse: int, dO: int, B: int, H: int, N: int, d: int,
+                      workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    return library().fa_bwd_preprocess(o, lse, dO, B, H, N, d, workspace,
+                                       int(workspace_bytes), stream or None)
+
+
+def fa_bwd_main(q: int, k: int, v: int, dO: int, dk: int, dv: int, B: int, H: int,
+                N: int, d: int, causal: int, scale: float, workspace: int,
+                workspace_bytes: int, stream: int = 0) -> int:
+    return library().fa_bwd_main(q, k, v, dO, dk, dv, B, H, N, d, int(causal),
+                                 float(scale), workspace, int(workspace_bytes),
+                                 stream or None)
+
+
+def fa_bwd_dq_convert(dq: int, B: int, H: int, N: int, d: int, scale: float,
+                      workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    return library().fa_bwd_dq_convert(dq, B, H, N, d, float(scale), workspace,
+                                       int(workspace_bytes), stream or None)
+
+
+def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(library().fa_bwd_workspace_size(B, H, N, d))
+
+
+def fa_get_device_error(stream: int = 0) -> int:
+    return library().fa_get_device_error(stream or None)
+
+
+# ---------------------------------------------------------------- tensor wrappers
+
+def _ptr(t: torch.Tensor) -> int:
+    return t.data_ptr()
+
+
+def _shape(q: torch.Tensor):
+    if q.dim() != 4:
+        raise ValueError("expected [B, H, N, d] tensors")
+    return tuple(q.shape)
+
+
+def _require(ts, shape, dtype, device):
+    for name, t in ts.items():
+        if t.dtype != dtype:
+            raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+        if t.device != device:
+            raise ValueError(f"{name}: expected device {device}, got {t.device}")
+        if not t.is_contiguous():
+            raise ValueError(f"{name}: must be contiguous")
+        if tuple(t.shape) != tuple(shape):
+            raise ValueError(f"{name}: expected shape {shape}, got {tuple(t.shape)}")
+
+
+def attention_forward(q, k, v, causal: bool, scale: float, out=None, lse=None,
+                      stream=None):
+    """O, LSE = fa_fwd(q, k, v) for CUDA bf16 [B,H,N,d] tensors."""
+    B, H, N, d = _shape(q)
+    _require({"q": q, "k": k, "v": v}, (B, H, N, d), torch.bfloat16, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _require({"out": out}, (B, H, N, d), torch.bfloat16, q.device)
+    _require({"lse": lse}, (B, H, N), torch.float32, q.device)
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    _check(fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d,
+                  int(causal), scale, s), "fa_fwd")
+    return out, lse
+
+
+def attention_backward(q, k, v, out, lse, dO, causal: bool, scale: float,
+                       dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV = fa_bwd(...) for CUDA bf16 [B,H,N,d] tensors."""
+    B, H, N, d = _shape(q)
+    _require({"q": q, "k": k, "v": v, "out": out, "dO": dO}, (B, H, N, d),
+             torch.bfloat16, q.device)
+    _require({"lse": lse}, (B, H, N), torch.float32, q.device)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(q) if dk is None else dk
+    dv = torch.empty_like(q) if dv is None else dv
+    _require({"dq": dq, "dk": dk, "dv": dv}, (B, H, N, d), torch.bfloat16,
+             q.device)
+    need = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    _check(fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(dO),
+                  _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, int(causal), scale,
+                  _ptr(workspace), workspace.numel() * workspace.element_size(),
+                  s), "fa_bwd")
+    return dq, dk, dv

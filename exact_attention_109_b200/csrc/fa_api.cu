@@ -1,0 +1,355 @@
+// fa_api.cu -- the C ABI of libfa_sm100.so (declared in include/fa.h):
+// argument checks, TMA tensor-map creation, kernel launches on the caller's
+// stream, and the per-device error word that bounded device waits write.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_bwd_kernels.cuh"
+#include "fa_fwd_kernel.cuh"
+
+// Set (bitwise OR) by a kernel whose pipeline wait ran out; one per device.
+__device__ unsigned int g_fa_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+struct DeviceState {
+    std::once_flag once;
+    bool ok = false;
+    unsigned int* err_word = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+
+bool load_encode() {
+    std::call_once(g_encode_once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// Opts the kernel into `bytes` of dynamic shared memory and checks that the
+// registers it is launched with cover its warpgroups' setmaxnreg split (an
+// increase beyond the launch allocation would never be granted).
+template <class K>
+bool prepare_kernel(K kernel, int bytes, int threads, int reg_budget) {
+    if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+        cudaSuccess)
+        return false;
+    cudaFuncAttributes attr{};
+    if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return false;
+    return attr.numRegs * threads >= reg_budget;
+}
+
+// One-time per-device set-up: architecture check, error-word address, and
+// the shared-memory opt-in of every kernel.  Returns FA_OK or an error.
+fa_status device_setup(int* dev_out, unsigned int** err_out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+    DeviceState& s = g_dev[dev];
+    std::call_once(s.once, [&] {
+        int major = 0;
+        if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) !=
+                cudaSuccess ||
+            major != 10)
+            return;
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_fa_error_word) != cudaSuccess) return;
+        s.err_word = static_cast<unsigned int*>(p);
+        bool ok = true;
+        ok &= prepare_kernel(fa::fa_fwd_kernel<64, false>, fa::FwdTraits<64>::SMEM_BYTES,
+                             fa::FwdTraits<64>::NUM_THREADS, fa::FwdTraits<64>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd_kernel<64, true>, fa::FwdTraits<64>::SMEM_BYTES,
+                             fa::FwdTraits<64>::NUM_THREADS, fa::FwdTraits<64>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd_kernel<128, false>, fa::FwdTraits<128>::SMEM_BYTES,
+                             fa::FwdTraits<128>::NUM_THREADS, fa::FwdTraits<128>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd_kernel<128, true>, fa::FwdTraits<128>::SMEM_BYTES,
+                             fa::FwdTraits<128>::NUM_THREADS, fa::FwdTraits<128>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_bwd_main_kernel<64, false>, fa::BwdTraits<64>::SMEM_BYTES,
+                             fa::BwdTraits<64>::NUM_THREADS, fa::BwdTraits<64>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_bwd_main_kernel<64, true>, fa::BwdTraits<64>::SMEM_BYTES,
+                             fa::BwdTraits<64>::NUM_THREADS, fa::BwdTraits<64>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_bwd_main_kernel<128, false>, fa::BwdTraits<128>::SMEM_BYTES,
+                             fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_bwd_main_kernel<128, true>, fa::BwdTraits<128>::SMEM_BYTES,
+                             fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
+        s.ok = ok;
+    });
+    if (!s.ok) {
+        int major = 0;
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        cudaGetLastError();
+        return major == 10 ? FA_ERR_CUDA : FA_ERR_UNSUPPORTED;
+    }
+    *dev_out = dev;
+    *err_out = s.err_word;
+    return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_sizes(int B, int H, int N, int d, float scale) {
+    if (B < 1 || H < 1 || N < 1) return FA_ERR_INVALID_ARG;
+    if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    const long long bh = static_cast<long long>(B) * H;
+    // TMA coordinates and row indices are 32-bit; keep every index in range.
+    if (bh > (1ll << 24) || N > (1 << 30) || bh * ((N + 255) / 256) > 0x7fffffffll)
+        return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
+// 3-D view [BH][rows][cols] of a row-major tensor, 128-byte swizzled boxes of
+// {box_cols, box_rows, 1}.
+bool encode_3d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+               int cols, long long rows, long long bh, int box_cols, int box_rows) {
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(bh)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * elem_bytes,
+                             static_cast<cuuint64_t>(rows) * cols * elem_bytes};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows), 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return g_encode(map, dtype, 3, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool encode_bf16(CUtensorMap* map, const void* base, int d, int N, long long bh, int box_rows) {
+    return encode_3d(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, box_rows);
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                       const CUtensorMap& mo, const fa::FwdParams& prm, long long bh,
+                       cudaStream_t stream) {
+    using T = fa::FwdTraits<D>;
+    const long long grid = bh * prm.n_qpairs;
+    fa::fa_fwd_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), T::NUM_THREADS, T::SMEM_BYTES,
+                                   stream>>>(mq, mk, mv, mo, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_strerror(fa_status s) {
+    switch (s) {
+        case FA_OK: return "FA_OK";
+        case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+        case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported head dim or device";
+        case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: pointer not 16-byte aligned";
+        case FA_ERR_CUDA: return "FA_ERR_CUDA: CUDA call failed";
+        case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: device pipeline wait ran out";
+    }
+    return "unknown fa_status";
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int N, int d, int causal, float scale, void* stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    fa_status st = check_sizes(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_MISALIGNED;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    int dev;
+    unsigned int* err;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    if (!load_encode()) return FA_ERR_CUDA;
+
+    const long long bh = static_cast<long long>(B) * H;
+    CUtensorMap mq, mk, mv, mo;
+    if (!encode_bf16(&mq, q, d, N, bh, 128) || !encode_bf16(&mk, k, d, N, bh, 128) ||
+        !encode_bf16(&mv, v, d, N, bh, 128) || !encode_bf16(&mo, o, d, N, bh, 32))
+        return FA_ERR_CUDA;
+    fa::FwdParams prm;
+    prm.lse = lse;
+    prm.err = err;
+    prm.N = N;
+    prm.n_qpairs = (N + 255) / 256;
+    prm.bh_count = static_cast<int>(bh);
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (d == 64)
+        e = causal ? launch_fwd<64, true>(mq, mk, mv, mo, prm, bh, s)
+                   : launch_fwd<64, false>(mq, mk, mv, mo, prm, bh, s);
+    else
+        e = causal ? launch_fwd<128, true>(mq, mk, mv, mo, prm, bh, s)
+                   : launch_fwd<128, false>(mq, mk, mv, mo, prm, bh, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+    if (check_sizes(B, H, N, d, 1.0f) != FA_OK) return 0;
+    return fa::bwd_workspace_bytes(static_cast<long long>(B) * H, N, d);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Checks shared by the backward stages; on success fills the workspace view.
+fa_status bwd_common(int B, int H, int N, int d, float scale, void* workspace,
+                     size_t workspace_bytes, fa::BwdWorkspace* ws, int* dev,
+                     unsigned int** err) {
+    if (!workspace) return FA_ERR_INVALID_ARG;
+    fa_status st = check_sizes(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    const long long bh = static_cast<long long>(B) * H;
+    if (workspace_bytes < fa::bwd_workspace_bytes(bh, N, d)) return FA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_MISALIGNED;
+    *ws = fa::bwd_workspace_layout(workspace, bh, N, d);
+    return FA_OK;
+}
+
+fa_status bwd_pre_impl(const void* o, const float* lse, const void* dO, int B, int H, int N,
+                       int d, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!o || !lse || !dO) return FA_ERR_INVALID_ARG;
+    fa::BwdWorkspace ws;
+    int dev;
+    unsigned int* err;
+    fa_status st = bwd_common(B, H, N, d, 1.0f, workspace, workspace_bytes, &ws, &dev, &err);
+    if (st != FA_OK) return st;
+    if (!aligned16(o) || !aligned16(lse) || !aligned16(dO)) return FA_ERR_MISALIGNED;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    const int bh = B * H;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = d == 64 ? fa::launch_bwd_pre<64>(o, lse, dO, bh, N, ws, s)
+                                  : fa::launch_bwd_pre<128>(o, lse, dO, bh, N, ws, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, void* dk,
+                        void* dv, int B, int H, int N, int d, int causal, float scale,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !dO || !dk || !dv) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    fa::BwdWorkspace ws;
+    int dev;
+    unsigned int* err;
+    fa_status st = bwd_common(B, H, N, d, scale, workspace, workspace_bytes, &ws, &dev, &err);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk) ||
+        !aligned16(dv))
+        return FA_ERR_MISALIGNED;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    if (!load_encode()) return FA_ERR_CUDA;
+    const long long bh = static_cast<long long>(B) * H;
+    CUtensorMap mq, mk, mv, mdo, mdk, mdv, macc;
+    if (!encode_bf16(&mq, q, d, N, bh, fa::kBwdBM) || !encode_bf16(&mk, k, d, N, bh, 128) ||
+        !encode_bf16(&mv, v, d, N, bh, 128) || !encode_bf16(&mdo, dO, d, N, bh, fa::kBwdBM) ||
+        !encode_bf16(&mdk, dk, d, N, bh, 32) || !encode_bf16(&mdv, dv, d, N, bh, 32) ||
+        !encode_3d(&macc, ws.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, ws.n_pad, bh, 32,
+                   fa::kBwdBM))
+        return FA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int ibh = static_cast<int>(bh);
+    cudaError_t e;
+    if (d == 64)
+        e = causal ? fa::launch_bwd_main<64, true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                   macc, err, s)
+                   : fa::launch_bwd_main<64, false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                    macc, err, s);
+    else
+        e = causal ? fa::launch_bwd_main<128, true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                    macc, err, s)
+                   : fa::launch_bwd_main<128, false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk,
+                                                     mdv, macc, err, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status bwd_convert_impl(void* dq, int B, int H, int N, int d, float scale, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    if (!dq) return FA_ERR_INVALID_ARG;
+    fa::BwdWorkspace ws;
+    int dev;
+    unsigned int* err;
+    fa_status st = bwd_common(B, H, N, d, scale, workspace, workspace_bytes, &ws, &dev, &err);
+    if (st != FA_OK) return st;
+    if (!aligned16(dq)) return FA_ERR_MISALIGNED;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int bh = B * H;
+    const cudaError_t e = d == 64 ? fa::launch_bwd_convert<64>(dq, bh, N, scale, ws, s)
+                                  : fa::launch_bwd_convert<128>(dq, bh, N, scale, ws, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_bwd_preprocess(const void* o, const float* lse, const void* dO, int B, int H, int N,
+                            int d, void* workspace, size_t workspace_bytes, void* stream) {
+    return bwd_pre_impl(o, lse, dO, B, H, N, d, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_main(const void* q, const void* k, const void* v, const void* dO, void* dk,
+                      void* dv, int B, int H, int N, int d, int causal, float scale,
+                      void* workspace, size_t workspace_bytes, void* stream) {
+    return bwd_main_impl(q, k, v, dO, dk, dv, B, H, N, d, causal, scale, workspace,
+                         workspace_bytes, stream);
+}
+
+fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+    return bwd_convert_impl(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+    // Validate everything before the first launch, so a failure enqueues nothing.
+    if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !workspace)
+        return FA_ERR_INVALID_ARG;
+    fa_status st = check_sizes(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (workspace_bytes < fa::bwd_workspace_bytes(static_cast<long long>(B) * H, N, d))
+        return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return FA_ERR_MISALIGNED;
+    int dev;
+    unsigned int* err;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    if (!load_encode()) return FA_ERR_CUDA;
+    if ((st = bwd_pre_impl(o, lse, dO, B, H, N, d, workspace, workspace_bytes, stream)) != FA_OK)
+        return st;
+    if ((st = bwd_main_impl(q, k, v, dO, dk, dv, B, H, N, d, causal, scale, workspace,
+                            workspace_bytes, stream)) != FA_OK)
+        return st;
+    return bwd_convert_impl(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_get_device_error(void* stream) {
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
+    unsigned int word = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&word, g_fa_error_word, sizeof(word)) != cudaSuccess)
+        return FA_ERR_CUDA;
+    if (word != 0 && cudaMemcpyToSymbol(g_fa_error_word, &zero, sizeof(zero)) != cudaSuccess)
+        return FA_ERR_CUDA;
+    return (word & fa::kErrTimeout) ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,409 @@
+// fa_fwd_kernel.cuh -- forward pass of exact attention for sm_100a.
+//
+// What it computes (FlashAttention-2 abstract; iplexlaw FlashAttention-2
+// blog, "Tiling preserves the attention calculation"): for every query row i,
+// O_i = sum_j softmax_j(scale * q_i.k_j) v_j over the visible keys, and the
+// row's log-sum-exp.  K and V stream through shared memory in 128-row blocks
+// while an online softmax keeps a running maximum m and sum l per row and
+// rescales the partial output, so the N x N scores never leave the SM.
+//
+// How it maps onto B200:
+//  * One CTA owns two 128-row query tiles of one (batch, head) and walks the
+//    key blocks once for both, so each K/V block fetched from L2/HBM feeds two
+//    tiles of MMAs (the pages' "split Q, share K/V" idea at CTA granularity).
+//  * Warp roles: warps 0-3 and 4-7 are the softmax warpgroups of tile 0 and
+//    tile 1 (one thread per query row, which is also its TMEM lane); warp 8
+//    issues tcgen05.mma from one thread; warp 9 issues TMA loads.
+//  * TMEM (512 columns): S/P of tile t at columns [128t, 128t+128), the O
+//    accumulator of tile t at [256 + d t, 256 + d t + d).  P is written back
+//    as bf16 over the first 64 columns of S and read by the PV MMA straight
+//    from TMEM.
+//  * K and V blocks share one ring of shared-memory slots (order K0, V0, K1,
+//    V1, ...) guarded by full/empty mbarriers; TMA zero-fills rows past N.
+//  * Fewer non-matmul operations (blog, "Three changes improve GPU
+//    utilisation"): the scale is folded into one FFMA before exp2, O is
+//    rescaled only when a row's maximum grows by more than 2^8 (the stale
+//    maximum is exact for the final result because l and O share it), and
+//    only the diagonal block and the ragged last block are masked; causal
+//    blocks above the diagonal are never loaded.
+#pragma once
+
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+template <int D>
+struct FwdTraits {
+    static_assert(D == 64 || D == 128, "head dim");
+    static constexpr int BM = 128;                  // query rows per tile
+    static constexpr int BN = 128;                  // key rows per block
+    static constexpr int TILES = 2;                 // query tiles per CTA
+    static constexpr int CHUNKS = D / 64;           // 128-byte swizzle column chunks
+    static constexpr int CHUNK_BYTES = 128 * 128;   // 128 rows x 128 B
+    static constexpr int TILE_BYTES = BM * D * 2;   // one 128-row bf16 tile
+    static constexpr int NSLOT = (D == 128) ? 4 : 8;
+    static constexpr int Q_OFF = 0;
+    static constexpr int KV_OFF = Q_OFF + TILES * TILE_BYTES;
+    static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
+    // q, full[NSLOT], empty[NSLOT], s_full[2], p_ready[2], o_final[2], mma_done
+    static constexpr int NBAR = 1 + 2 * NSLOT + 2 + 2 + 2 + 1;
+    static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+    static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
+    static constexpr int NUM_THREADS = 384;  // 3 warpgroups; warps 10-11 idle
+    static constexpr int MMA_WARP = 8;
+    static constexpr int LOAD_WARP = 9;
+    // Register split: softmax warpgroups grow, the MMA/TMA warpgroup shrinks.
+    static constexpr uint32_t REG_SOFTMAX = 216;
+    static constexpr uint32_t REG_CONTROL = 72;
+    static constexpr int REG_BUDGET = 128 * (2 * REG_SOFTMAX + REG_CONTROL);
+    static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
+    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
+    static constexpr float TAU = 8.0f;  // deferred-rescale threshold (log2 units)
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+struct FwdParams {
+    float* lse;            // [BH, N]
+    unsigned int* err;     // device error word
+    int N;
+    int n_qpairs;          // ceil(N / 256)
+    int bh_count;          // B * H
+    float scale_log2;      // scale * log2(e)
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                  const FwdParams p) {
+    using T = FwdTraits<D>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + T::BAR_OFF);
+    uint64_t* bar_q = bars;
+    uint64_t* full = bars + 1;
+    uint64_t* empty = full + T::NSLOT;
+    uint64_t* s_full = empty + T::NSLOT;
+    uint64_t* p_ready = s_full + 2;
+    uint64_t* o_final = p_ready + 2;
+    uint64_t* mma_done = o_final + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::MISC_OFF);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::MISC_OFF + 4);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // Non-causal: consecutive CTAs share a head (K/V reuse in L2).  Causal:
+    // heavy tiles first -- the last query pair of every head has the most key
+    // blocks, so the grid walks query pairs from the end.
+    int qp, bh;
+    if (CAUSAL) {
+        bh = static_cast<int>(blockIdx.x % p.bh_count);
+        qp = p.n_qpairs - 1 - static_cast<int>(blockIdx.x / p.bh_count);
+    } else {
+        qp = static_cast<int>(blockIdx.x % p.n_qpairs);
+        bh = static_cast<int>(blockIdx.x / p.n_qpairs);
+    }
+    const int N = p.N;
+    const int q0 = qp * 256;
+    const int n_kv = (N + T::BN - 1) / T::BN;
+    const int n0 = CAUSAL ? min(n_kv, 2 * qp + 1) : n_kv;  // key blocks of tile 0
+    const int n1 = CAUSAL ? min(n_kv, 2 * qp + 2) : n_kv;  // key blocks of tile 1
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int s = 0; s < T::NSLOT; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(&s_full[t], 1);
+            mbar_init(&p_ready[t], 128);
+            mbar_init(&o_final[t], 1);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == T::MMA_WARP) {
+        tmem_alloc(tmem_slot, T::TMEM_COLS);
+        tmem_relinquish();
+    }
+    if (warp == T::LOAD_WARP && lane == 0) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
+        tma_prefetch_desc(&tmO);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const AbortState st{abort_flag, p.err};
+    if (warp >= 8) {
+      setmaxnreg_dec<T::REG_CONTROL>();
+      if (warp == T::LOAD_WARP) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            bool ok = true;
+            mbar_arrive_expect_tx(bar_q, T::TILES * T::TILE_BYTES);
+            for (int t = 0; t < T::TILES; ++t)
+                for (int c = 0; c < T::CHUNKS; ++c)
+                    tma_load_3d(smem + T::Q_OFF + t * T::TILE_BYTES + c * T::CHUNK_BYTES, &tmQ,
+                                bar_q, c * 64, q0 + 128 * t, bh);
+            int issued = 0;
+            for (int j = 0; j < n1 && ok; ++j) {
+                for (int h = 0; h < 2; ++h) {  // 0: K_j, 1: V_j
+                    const int idx = 2 * j + h;
+                    const int slot = idx % T::NSLOT;
+                    const uint32_t par = (idx / T::NSLOT) & 1;
+                    if (!mbar_wait(&empty[slot], par ^ 1u, st)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&full[slot], T::TILE_BYTES);
+                    uint8_t* dst = smem + T::KV_OFF + slot * T::TILE_BYTES;
+                    for (int c = 0; c < T::CHUNKS; ++c)
+                        tma_load_3d(dst + c * T::CHUNK_BYTES, h ? &tmV : &tmK, &full[slot], c * 64,
+                                    j * T::BN, bh);
+                    ++issued;
+                }
+            }
+            if (!ok) {
+                // Let copies still in flight land before the CTA exits.
+                for (int idx = max(0, issued - T::NSLOT); idx < issued; ++idx)
+                    mbar_wait_bounded(&full[idx % T::NSLOT], (idx / T::NSLOT) & 1);
+                mbar_wait_bounded(bar_q, 0);
+            }
+        }
+        __syncwarp();
+      } else if (warp == T::MMA_WARP) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t q_base = smem_u32(smem + T::Q_OFF);
+            const uint32_t kv_base = smem_u32(smem + T::KV_OFF);
+            auto slot_addr = [&](int idx) {
+                return kv_base + static_cast<uint32_t>((idx % T::NSLOT) * T::TILE_BYTES);
+            };
+            auto slot_par = [&](int idx) { return static_cast<uint32_t>((idx / T::NSLOT) & 1); };
+            // S_t = Q_t K^T : M=128, N=128, K=D, both operands K-major.
+            auto mma_s = [&](int t, uint32_t k_addr) {
+#pragma unroll
+                for (int k = 0; k < D / 16; ++k) {
+                    const uint32_t off = (k >> 2) * T::CHUNK_BYTES + (k & 3) * 32;
+                    const uint64_t a = sdesc_sw128(q_base + t * T::TILE_BYTES + off, 16, 1024);
+                    const uint64_t b = sdesc_sw128(k_addr + off, 16, 1024);
+                    umma_ss(tmem + 128u * t, a, b, T::IDESC_S, k > 0 ? 1u : 0u);
+                }
+            };
+            // O_t += P_t V : M=128, N=D, K=128; P from TMEM, V MN-major.
+            auto mma_pv = [&](int t, uint32_t v_addr, bool accumulate) {
+#pragma unroll
+                for (int k = 0; k < T::BN / 16; ++k) {
+                    const uint64_t b = sdesc_sw128(v_addr + k * 2048, T::CHUNK_BYTES, 1024);
+                    umma_ts(tmem + 256u + D * t, tmem + 128u * t + 8u * k, b, T::IDESC_PV,
+                            (accumulate || k > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = mbar_wait(bar_q, 0, st) && mbar_wait(&full[0], 0, st);
+            if (ok) {
+                tc_fence_after();
+                mma_s(0, slot_addr(0));
+                umma_commit(&s_full[0]);
+                mma_s(1, slot_addr(0));
+                umma_commit(&s_full[1]);
+                umma_commit(&empty[0]);
+            }
+            for (int j = 1; j < n1 && ok; ++j) {
+                const int ik = 2 * j, iv = 2 * j - 1;  // K_j and V_{j-1}
+                ok = mbar_wait(&full[ik % T::NSLOT], slot_par(ik), st) &&
+                     mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st);
+                if (!ok) break;
+                tc_fence_after();
+                if (j - 1 < n0) {
+                    if (!(ok = mbar_wait(&p_ready[0], (j - 1) & 1, st))) break;
+                    tc_fence_after();
+                    mma_pv(0, slot_addr(iv), j - 1 > 0);
+                    if (j - 1 == n0 - 1) umma_commit(&o_final[0]);
+                }
+                if (j < n0) {
+                    mma_s(0, slot_addr(ik));
+                    umma_commit(&s_full[0]);
+                }
+                if (!(ok = mbar_wait(&p_ready[1], (j - 1) & 1, st))) break;
+                tc_fence_after();
+                mma_pv(1, slot_addr(iv), j - 1 > 0);
+                umma_commit(&empty[iv % T::NSLOT]);
+                mma_s(1, slot_addr(ik));
+                umma_commit(&s_full[1]);
+                umma_commit(&empty[ik % T::NSLOT]);
+            }
+            if (ok) {
+                const int jl = n1 - 1, iv = 2 * n1 - 1;
+                ok = mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st);
+                if (ok && jl < n0) {
+                    ok = mbar_wait(&p_ready[0], jl & 1, st);
+                    if (ok) {
+                        tc_fence_after();
+                        mma_pv(0, slot_addr(iv), jl > 0);
+                        umma_commit(&o_final[0]);
+                    }
+                }
+                if (ok) ok = mbar_wait(&p_ready[1], jl & 1, st);
+                if (ok) {
+                    tc_fence_after();
+                    mma_pv(1, slot_addr(iv), jl > 0);
+                    umma_commit(&o_final[1]);
+                    umma_commit(&empty[iv % T::NSLOT]);
+                }
+            }
+            // No MMA may still be running when TMEM is released.
+            umma_commit(mma_done);
+            mbar_wait_bounded(mma_done, 0);
+        }
+        __syncwarp();
+      }
+    } else {
+        // ------------------------------------------------ softmax warpgroups
+        setmaxnreg_inc<T::REG_SOFTMAX>();
+        const int t = warp >> 2;         // query tile
+        const int lg = warp & 3;         // TMEM lane group of this warp
+        const int r = lg * 32 + lane;    // row within the tile = TMEM lane
+        const int row0 = q0 + 128 * t;
+        const int row = row0 + r;
+        const int nt = t ? n1 : n0;
+        const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
+        const uint32_t s_tm = tmem + lane_off + 128u * t;
+        const uint32_t o_tm = tmem + lane_off + 256u + D * t;
+        const float sl2 = p.scale_log2;
+        float m = -INFINITY;  // reference maximum, log2 units of scaled scores
+        float l = 0.f;        // running sum of exp2(score - m), fp32 (for LSE)
+        float lr = 0.f;       // the same sum over the bf16-rounded weights the
+                              // PV MMA uses (normalises O consistently)
+        bool ok = true;
+
+        for (int j = 0; j < nt; ++j) {
+            ok = __all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1, st));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sr[4][32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + 32u * c, sr[c]);
+            tmem_ld_wait();
+
+            const int kv0 = j * T::BN;
+            int lim = T::BN;
+            if (kv0 + T::BN > N) lim = N - kv0;
+            if (CAUSAL && kv0 + T::BN - 1 > row0) lim = min(lim, row - kv0 + 1);
+            if (lim < T::BN) {
+#pragma unroll
+                for (int c = 0; c < 128; ++c)
+                    if (c >= lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
+            }
+            float mx0 = __uint_as_float(sr[0][0]), mx1 = __uint_as_float(sr[0][1]);
+#pragma unroll
+            for (int c = 2; c < 128; c += 2) {
+                mx0 = fmaxf(mx0, __uint_as_float(sr[c >> 5][c & 31]));
+                mx1 = fmaxf(mx1, __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]));
+            }
+            const float m_blk = fmaxf(mx0, mx1) * sl2;
+            const float m_new = (m_blk > m + T::TAU) ? m_blk : m;
+            if (j > 0) {
+                const bool grow = m_new != m;
+                if (__any_sync(0xffffffffu, grow)) {
+                    const float alpha = grow ? ex2_approx(m - m_new) : 1.0f;
+                    l *= alpha;
+                    lr *= alpha;
+#pragma unroll 1
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t o[32];
+                        tmem_ld32(o_tm + 32u * c, o);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tmem_st32(o_tm + 32u * c, o);
+                    }
+                }
+            }
+            m = m_new;
+            const float neg_m = -m;
+            float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int c = 64 * h + 2 * e;
+                    const float p0 =
+                        ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), sl2, neg_m));
+                    const float p1 = ex2_approx(
+                        fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), sl2, neg_m));
+                    sum0 += p0;
+                    sum1 += p1;
+                    pk[e] = pack_bf16x2(p0, p1);
+                    rsum0 += __uint_as_float(pk[e] << 16);
+                    rsum1 += __uint_as_float(pk[e] & 0xffff0000u);
+                }
+                tmem_st32(s_tm + 32u * h, pk);
+            }
+            l += sum0 + sum1;
+            lr += rsum0 + rsum1;
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&p_ready[t]);
+        }
+
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0, st));
+        if (ok) {
+            tc_fence_after();
+            const float inv_l = 1.0f / lr;
+            const float lse_val = (m + log2f(l)) * 0.6931471805599453f;
+            // Stage O (bf16, 128-byte swizzle) in this tile's Q buffer, which
+            // no MMA reads any more, then store this warp's 32 rows by TMA.
+            uint8_t* stage = smem + T::Q_OFF + t * T::TILE_BYTES + lg * 32 * 128;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tmem_ld32(o_tm + 32u * c, o);
+                tmem_ld_wait();
+                uint8_t* chunk = stage + (c >> 1) * T::CHUNK_BYTES;
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(o[8 * u + 0]) * inv_l,
+                                      __uint_as_float(o[8 * u + 1]) * inv_l);
+                    v.y = pack_bf16x2(__uint_as_float(o[8 * u + 2]) * inv_l,
+                                      __uint_as_float(o[8 * u + 3]) * inv_l);
+                    v.z = pack_bf16x2(__uint_as_float(o[8 * u + 4]) * inv_l,
+                                      __uint_as_float(o[8 * u + 5]) * inv_l);
+                    v.w = pack_bf16x2(__uint_as_float(o[8 * u + 6]) * inv_l,
+                                      __uint_as_float(o[8 * u + 7]) * inv_l);
+                    *reinterpret_cast<uint4*>(chunk + sw128_offset(lane, (c & 1) * 4 + u)) = v;
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            const int wrow0 = row0 + lg * 32;
+            if (lane == 0 && wrow0 < N) {
+                for (int c = 0; c < T::CHUNKS; ++c)
+                    tma_store_3d(&tmO, stage + c * T::CHUNK_BYTES, c * 64, wrow0, bh);
+                bulk_commit_group();
+                bulk_wait_group_read0();
+            }
+            if (row < N) p.lse[static_cast<size_t>(bh) * N + row] = lse_val;
+        }
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == T::MMA_WARP) {
+        tc_fence_after();
+        tmem_dealloc(tmem, T::TMEM_COLS);
+    }
+}
+
+}  // namespace fa

@@ -1,0 +1,151 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library, libfa_sm100.so.
+ *
+ * The library computes exact scaled-dot-product attention
+ *
+ *     O = softmax(scale * Q K^T [+ causal mask]) V
+ *
+ * and its gradient, tile by tile with an online softmax, so that the N x N
+ * score and probability matrices never reach HBM.  Sources:
+ *   - "FlashAttention-2: Faster Attention with Better Parallelism and Work
+ *     Partitioning" (abstract): exact attention, no approximation; memory
+ *     linear in the sequence length; work split over sequence, batch and heads.
+ *   - iplexlaw blog "FlashAttention-2 GPU work partitioning", section "Tiling
+ *     preserves the attention calculation": tiles are staged on chip and an
+ *     online softmax rescales running statistics and partial outputs so the
+ *     blocks add up to the globally normalised result; section "Three changes
+ *     improve GPU utilisation": fewer non-matmul operations (rescaling, bounds
+ *     and causal-mask handling), parallelism along the sequence dimension.
+ * The log-sum-exp output and the backward algorithm (recompute P from LSE,
+ * D = rowsum(dO * O), fp32 reduction of dQ) are the standard gradient of the
+ * definition; the pages name gradients and training but print no formula.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are contiguous row-major [B, H, N, d] in bf16 (Q, K, V, O, dO,
+ *     dQ, dK, dV); row (b, h, n) starts at element ((b*H + h)*N + n)*d.
+ *     LSE is [B, H, N] fp32.  N_q = N_k = N.
+ *   - Every pointer is a DEVICE pointer on the current CUDA device, 16-byte
+ *     aligned (TMA requirement).  The caller owns every buffer; the library
+ *     allocates no device memory and keeps no state beyond a per-device error
+ *     word and one-time kernel attributes.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; no call synchronises the
+ *     host except fa_get_device_error.
+ *   - A status other than FA_OK means nothing was enqueued.
+ *   - Supported: d in {64, 128}; N >= 1; B, H >= 1; B*H*N*d < 2^31 rows*cols
+ *     per tensor index space of one head batch; scale finite and > 0.
+ *     causal: key j is visible to query i iff j <= i.
+ *   - Device-side waits are bounded (about 2 s).  A kernel whose pipeline wait
+ *     runs out records FA_ERR_TIMEOUT in the device error word and returns
+ *     early; fa_get_device_error reports it.
+ */
+#ifndef FA_SM100_H
+#define FA_SM100_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FA_OK = 0,
+    FA_ERR_INVALID_ARG = 1,  /* null pointer, bad size, non-finite/<=0 scale */
+    FA_ERR_UNSUPPORTED = 2,  /* d not in {64,128}, or no sm_100 device       */
+    FA_ERR_MISALIGNED = 3,   /* a pointer is not 16-byte aligned             */
+    FA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed            */
+    FA_ERR_TIMEOUT = 5       /* a device-side pipeline wait ran out          */
+} fa_status;
+
+/*
+ * fa_fwd -- forward pass.
+ *   q, k, v  [B,H,N,d] bf16, read only.
+ *   o        [B,H,N,d] bf16, written: O_i = sum_j P_ij v_j.
+ *   lse      [B,H,N] fp32, written: LSE_i = ln sum_{j visible} exp(scale q_i.k_j)
+ *            (natural log), the statistic fa_bwd consumes.
+ *   causal   0 or 1.  scale: multiplies Q K^T (commonly 1/sqrt(d)).
+ * Cites: FlashAttention-2 abstract (exact attention, tiled, sequence-parallel);
+ * iplexlaw blog, "Tiling preserves the attention calculation" (online softmax).
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_MISALIGNED,
+ * FA_ERR_CUDA (launch failure).  o and lse may not alias the inputs.
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o,
+                 float* lse, int B, int H, int N, int d, int causal,
+                 float scale, void* stream);
+
+/*
+ * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs:
+ * an fp32 dQ accumulator [B,H,Npad,d] plus two fp32 row vectors [B,H,Npad]
+ * (log2-scaled LSE and D = rowsum(dO * O)), Npad = N rounded up to 128.
+ * Linear in N (FlashAttention-2 abstract: memory linear, not quadratic).
+ * Returns 0 for invalid sizes.
+ */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * fa_bwd -- backward pass.
+ *   q, k, v, o, lse   as passed to / produced by one fa_fwd call (same
+ *                     causal and scale).
+ *   dO                [B,H,N,d] bf16 upstream gradient, read only.
+ *   dq, dk, dv        [B,H,N,d] bf16, overwritten (not accumulated).
+ *   workspace         device buffer of >= fa_bwd_workspace_size(B,H,N,d)
+ *                     bytes, 256-byte aligned; contents need no
+ *                     initialisation and are clobbered.
+ * Three launches on `stream`: preprocess (D, log2 LSE, zero dQ accumulator),
+ * the main kernel (one CTA per key block; recomputes P from LSE; dK, dV per
+ * key block; dQ by fp32 reduction), and the dQ conversion to bf16.
+ * dQ is not bitwise deterministic (fp32 reduction order varies); dK and dV are.
+ * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG when the workspace is too small.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
+                 const float* lse, const void* dO, void* dq, void* dk,
+                 void* dv, int B, int H, int N, int d, int causal, float scale,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The three stages fa_bwd runs, callable one by one on the same workspace
+ * (for example to time the main kernel alone).  Same conventions as fa_bwd;
+ * each returns FA_OK after enqueueing its launch.
+ *
+ * fa_bwd_preprocess -- D_i = sum_d dO_id * O_id (fp32), LSE_i * log2(e), and a
+ *   zeroed fp32 dQ accumulator, all in `workspace`.  Reads o, lse, dO.
+ */
+fa_status fa_bwd_preprocess(const void* o, const float* lse, const void* dO,
+                            int B, int H, int N, int d, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * fa_bwd_main -- one CTA per (b, h, 128-row key block): recomputes P from the
+ *   stored LSE, writes dK (times scale) and dV in bf16, and reduce-adds the
+ *   unscaled dQ into the workspace accumulator.  Needs fa_bwd_preprocess's
+ *   workspace contents.
+ */
+fa_status fa_bwd_main(const void* q, const void* k, const void* v,
+                      const void* dO, void* dk, void* dv, int B, int H, int N,
+                      int d, int causal, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
+ * fa_bwd_dq_convert -- dq = bf16(scale * accumulator).  Needs fa_bwd_main's
+ *   workspace contents.
+ */
+fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale,
+                            void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
+ * fa_get_device_error -- synchronises `stream`, then reads and clears the
+ * current device's error word.  Returns FA_ERR_TIMEOUT if a kernel's bounded
+ * pipeline wait ran out since the last call, FA_ERR_CUDA if the stream
+ * reports a CUDA error, FA_OK otherwise.
+ */
+fa_status fa_get_device_error(void* stream);
+
+/* fa_strerror -- static, human-readable name of a status. */
+const char* fa_strerror(fa_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_SM100_H */
