@@ -253,6 +253,31 @@ def reference_arm(args, w, wname):
     return 0
 
 
+def shard_heads(heads_per_rank: int, world: int, rank: int):
+    """Global head range [start, stop) that `rank` owns when every rank runs
+    its own heads_per_rank independent heads (weak scaling: the per-GPU work
+    is fixed, the global problem grows with the number of ranks)."""
+    start = rank * heads_per_rank
+    return start, start + heads_per_rank
+
+
+def max_over_ranks(value_ms: float, device=None) -> float:
+    """The slowest rank's time (max-reduce when a process group is active)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value_ms)], dtype=torch.float64,
+                     device=device if device is not None else "cpu")
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank_step: float, steps: int, world: int,
+                   max_ms: float) -> float:
+    """Whole-job TFLOP/s: the work of all ranks over the slowest rank's time."""
+    return flops_per_rank_step * steps * world / (max_ms * 1e-3) / 1e12
+
+
 def workload_config(w, wname):
     return {"workload": wname, "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
             "causal": w["causal"], "inputs": w["dist"], "pass": "fwd+bwd",
@@ -281,7 +306,8 @@ def gpu_arm(args, w, wname):
 
     B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
     scale = default_scale(d)
-    host = attention_inputs(B, H, N, d, w["seed"] + rank, w["dist"], with_dout=True)
+    head0, _ = shard_heads(B * H, world, rank)
+    host = attention_inputs(B, H, N, d, w["seed"] + head0, w["dist"], with_dout=True)
     dev = {k_: v_.cuda() for k_, v_ in host.items()}
     q, k, v, dO = dev["q"], dev["k"], dev["v"], dev["dO"]
     o = torch.empty_like(q)
@@ -351,13 +377,9 @@ def gpu_arm(args, w, wname):
     elapsed_ms = evs[0][0].elapsed_time(evs[-1][-1])
     per_stage = [sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
                  for j in range(len(stages))]
-    t = torch.tensor([elapsed_ms], dtype=torch.float64, device=q.device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    elapsed_max = float(t.item())
-
+    elapsed_max = max_over_ranks(elapsed_ms, q.device)
     flops_step = 3.5 * fwd_flops(w)
-    value = flops_step * K * world / (elapsed_max * 1e-3) / 1e12
+    value = job_throughput(flops_step, K, world, elapsed_max)
 
     # ---- end to end through the public API with pinned host buffers
     pin = {x: host[x].pin_memory() for x in ("q", "k", "v", "dO")}
@@ -387,10 +409,8 @@ def gpu_arm(args, w, wname):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=q.device)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_value = flops_step * Ke * world / (float(te.item()) * 1e-3) / 1e12
+    e2e_value = job_throughput(flops_step, Ke, world,
+                               max_over_ranks(e0.elapsed_time(e1), q.device))
     status = fa.fa_get_device_error()
     if status != fa.FA_OK:
         raise fa.FaError(status, "e2e")
