@@ -60,6 +60,9 @@ def library():
     lib.fa_bwd_main.restype = i
     lib.fa_bwd_dq_convert.argtypes = [vp, i, i, i, i, f, vp, sz, vp]
     lib.fa_bwd_dq_convert.restype = i
+    lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f,
+                                   vp]
+    lib.fa_bwd_noalloc.restype = i
     lib.fa_get_device_error.argtypes = [vp]
     lib.fa_get_device_error.restype = i
     lib.fa_strerror.argtypes = [i]
@@ -113,6 +116,20 @@ def fa_bwd_dq_convert(dq: int, B: int, H: int, N: int, d: int, scale: float,
                       workspace: int, workspace_bytes: int, stream: int = 0) -> int:
     return library().fa_bwd_dq_convert(dq, B, H, N, d, float(scale), workspace,
                                        int(workspace_bytes), stream or None)
+
+
+def fa_bwd_noalloc(q: int, k: int, v: int, o: int, lse: int, dO: int, dq: int,
+                   dk: int, dv: int, B: int, H: int, N: int, d: int, causal: int,
+                   scale: float, stream: int = 0) -> int:
+    """Raw C call of the backward pass that uses the library's own fixed scratch
+    array instead of a caller workspace (for callers that cannot allocate);
+    returns the status."""
+    return library().fa_bwd_noalloc(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d,
+                                    int(causal), float(scale), stream or None)
+
+
+# Size of the scratch array fa_bwd_noalloc uses (FA_BWD_NOALLOC_MAX_WORKSPACE_BYTES).
+FA_BWD_NOALLOC_MAX_WORKSPACE_BYTES = 64 << 20
 
 
 def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:

@@ -7,7 +7,8 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SOURCES = [os.path.join(HERE, "csrc", "fa_api.cu")]
+SOURCES = [os.path.join(HERE, "csrc", "fa_api.cu"),
+           os.path.join(HERE, "csrc", "fa_noalloc.cu")]
 HEADERS = [os.path.join(HERE, "csrc", f) for f in
            ("sm100_ptx.cuh", "fa_fwd_kernel.cuh", "fa_bwd_kernels.cuh")] + \
           [os.path.join(ROOT, "include", "fa.h")]

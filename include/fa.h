@@ -134,6 +134,36 @@ fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale,
                             void* stream);
 
 /*
+ * fa_bwd_noalloc -- fa_bwd for callers that cannot allocate device memory.
+ * (No counterpart in the paper; it is a packaging choice of this library.)
+ *   Some callers have no way to hand fa_bwd a workspace: a plugin inside a host
+ *   application that owns all device memory through its own pool and gives
+ *   extensions no allocator, or a serving path that forbids cudaMalloc after
+ *   start-up because it can synchronise the device and take driver locks.
+ *   This entry point takes the same arguments as fa_bwd minus the workspace
+ *   and uses a fixed scratch array of FA_BWD_NOALLOC_MAX_WORKSPACE_BYTES that
+ *   the library reserves, at load, on every GPU that loads it (held until the
+ *   process exits).  It calls no allocator itself.
+ *   - Problems whose fa_bwd_workspace_size exceeds that maximum are rejected
+ *     with FA_ERR_INVALID_ARG before anything is enqueued (d outside {64, 128}
+ *     gives FA_ERR_UNSUPPORTED).
+ *   - The first call on a device looks up the scratch array's device address
+ *     (a one-time set-up per device, done with that device current); make
+ *     that first call before any stream capture.
+ *   - All calls on a device share the one array, which keeps whatever the
+ *     last call left in it; each call rewrites what it reads before reading
+ *     it.  Calls whose GPU work overlaps (e.g. on two streams without
+ *     ordering between them) race on the array and give wrong results:
+ *     order them on one stream or with events.
+ *   Other conventions, outputs and errors are those of fa_bwd.
+ */
+#define FA_BWD_NOALLOC_MAX_WORKSPACE_BYTES ((size_t)64 << 20)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
+                         const void* o, const float* lse, const void* dO,
+                         void* dq, void* dk, void* dv, int B, int H, int N,
+                         int d, int causal, float scale, void* stream);
+
+/*
  * fa_get_device_error -- synchronises `stream`, then reads and clears the
  * current device's error word.  Returns FA_ERR_TIMEOUT if a kernel's bounded
  * pipeline wait ran out since the last call, FA_ERR_CUDA if the stream
