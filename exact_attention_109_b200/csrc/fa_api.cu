@@ -349,7 +349,8 @@ fa_status fa_get_device_error(void* stream) {
         return FA_ERR_CUDA;
     if (word != 0 && cudaMemcpyToSymbol(g_fa_error_word, &zero, sizeof(zero)) != cudaSuccess)
         return FA_ERR_CUDA;
-    return (word & fa::kErrTimeout) ? FA_ERR_TIMEOUT : FA_OK;
+    if (word & fa::kErrTimeout) return FA_ERR_TIMEOUT;
+    return word ? FA_ERR_CUDA : FA_OK;
 }
 
 }  // extern "C"

@@ -207,10 +207,18 @@ __global__ void __launch_bounds__(384, 1) fa_bwd_main_kernel(
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    // Key block j of head bh; causal key blocks near the start see the most
-    // query blocks, so they come first.
-    const int j = static_cast<int>(blockIdx.x % p.n_kv);
-    const int bh = static_cast<int>(blockIdx.x / p.n_kv);
+    // Key block j of head bh.  Non-causal: a head's key blocks are adjacent
+    // (they share Q and dO in L2).  Causal: key block j walks n_q - 2j query
+    // blocks, so the grid takes every head's block 0 first, then every head's
+    // block 1, ... (longest first), which keeps a heavy CTA from starting last.
+    int j, bh;
+    if (CAUSAL) {
+        j = static_cast<int>(blockIdx.x / p.bh_count);
+        bh = static_cast<int>(blockIdx.x % p.bh_count);
+    } else {
+        j = static_cast<int>(blockIdx.x % p.n_kv);
+        bh = static_cast<int>(blockIdx.x / p.n_kv);
+    }
     const int N = p.N;
     const int qb0 = CAUSAL ? 2 * j : 0;   // first query block at/below the diagonal
     const int n = p.n_q - qb0;            // query blocks this CTA walks (>= 1)

@@ -72,6 +72,42 @@ struct FwdParams {
     float scale_log2;      // scale * log2(e)
 };
 
+// One softmax row over a 128-key block: p = exp2(s * scale*log2(e) - m) in
+// pairs (f32x2 FFMA for the argument), packed to bf16 and written over the
+// first 64 TMEM columns of S; returns the fp32 sum of p (for the LSE) and of
+// the bf16-rounded p (for normalising O) through two f32x2 accumulators each.
+__device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], float sl2,
+                                                  float m, uint32_t s_tm, float& l, float& lr) {
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    const uint64_t negm2 = f2_pack(-m, -m);
+    uint64_t sum2[2] = {0ull, 0ull}, rsum2[2] = {0ull, 0ull};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int c = 64 * h + 2 * e;
+            const uint64_t x2 = ffma2(f2_pack(__uint_as_float(sr[c >> 5][c & 31]),
+                                              __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31])),
+                                      sl2x2, negm2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            sum2[e & 1] = fadd2(sum2[e & 1], f2_pack(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
+            rsum2[e & 1] = fadd2(rsum2[e & 1], f2_pack(__uint_as_float(pk[e] << 16),
+                                                       __uint_as_float(pk[e] & 0xffff0000u)));
+        }
+        tmem_st32(s_tm + 32u * h, pk);
+    }
+    float a0, a1, b0, b1;
+    f2_unpack(fadd2(sum2[0], sum2[1]), a0, a1);
+    f2_unpack(fadd2(rsum2[0], rsum2[1]), b0, b1);
+    l += a0 + a1;
+    lr += b0 + b1;
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -294,21 +330,29 @@ __global__ void __launch_bounds__(384, 1)
             tmem_ld_wait();
 
             const int kv0 = j * T::BN;
-            int lim = T::BN;
-            if (kv0 + T::BN > N) lim = N - kv0;
-            if (CAUSAL && kv0 + T::BN - 1 > row0) lim = min(lim, row - kv0 + 1);
-            if (lim < T::BN) {
+            // Only the ragged last block and (causal) the diagonal block hold
+            // hidden scores; the test is uniform over the tile.
+            const bool masked_block =
+                (kv0 + T::BN > N) || (CAUSAL && kv0 + T::BN - 1 > row0);
+            if (masked_block) {
+                int lim = min(T::BN, N - kv0);
+                if (CAUSAL) lim = min(lim, row - kv0 + 1);
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (c >= lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
             }
-            float mx0 = __uint_as_float(sr[0][0]), mx1 = __uint_as_float(sr[0][1]);
+            // Row maximum: eight independent chains, then a tree.
+            float mx[8];
 #pragma unroll
-            for (int c = 2; c < 128; c += 2) {
-                mx0 = fmaxf(mx0, __uint_as_float(sr[c >> 5][c & 31]));
-                mx1 = fmaxf(mx1, __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]));
-            }
-            const float m_blk = fmaxf(mx0, mx1) * sl2;
+            for (int i = 0; i < 8; ++i) mx[i] = __uint_as_float(sr[0][i]);
+#pragma unroll
+            for (int c = 8; c < 128; c += 8)
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    mx[i] = fmaxf(mx[i], __uint_as_float(sr[(c + i) >> 5][(c + i) & 31]));
+            mx[0] = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                          fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float m_blk = mx[0] * sl2;
             const float m_new = (m_blk > m + T::TAU) ? m_blk : m;
             if (j > 0) {
                 const bool grow = m_new != m;
@@ -329,28 +373,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             m = m_new;
-            const float neg_m = -m;
-            float sum0 = 0.f, sum1 = 0.f, rsum0 = 0.f, rsum1 = 0.f;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                uint32_t pk[32];
-#pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int c = 64 * h + 2 * e;
-                    const float p0 =
-                        ex2_approx(fmaf(__uint_as_float(sr[c >> 5][c & 31]), sl2, neg_m));
-                    const float p1 = ex2_approx(
-                        fmaf(__uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31]), sl2, neg_m));
-                    sum0 += p0;
-                    sum1 += p1;
-                    pk[e] = pack_bf16x2(p0, p1);
-                    rsum0 += __uint_as_float(pk[e] << 16);
-                    rsum1 += __uint_as_float(pk[e] & 0xffff0000u);
-                }
-                tmem_st32(s_tm + 32u * h, pk);
-            }
-            l += sum0 + sum1;
-            lr += rsum0 + rsum1;
+            softmax_block_exp(sr, sl2, m, s_tm, l, lr);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_ready[t]);
