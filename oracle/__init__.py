@@ -56,6 +56,8 @@ def open_library(path: str):
     lib.ref_dkdv_rows.argtypes = [_D, _D, _D, _D, _D, _D, i, i, i, d, _LL, i,
                                   _D, _D]
     lib.ref_dkdv_rows.restype = None
+    lib.ref_fwd_decode.argtypes = [_D, _D, _D, _D, _D, i, i, i, i, i, d]
+    lib.ref_fwd_decode.restype = i
     lib.ref_num_threads.argtypes = []
     lib.ref_num_threads.restype = i
     return lib
@@ -176,3 +178,21 @@ def ref_dkdv_rows(q, k, v, dO, lse, D, rows, causal: bool, scale: float,
                       int(bool(causal)), float(scale), r.ctypes.data_as(_LL),
                       len(r), _p(dk), _p(dv))
     return dk, dv
+
+
+def ref_fwd_decode(q, k, v, causal: bool, scale: float, lib=None):
+    """O and LSE for Nq queries against Nk keys ([B,H,Nq,d] and [B,H,Nk,d]);
+    causal: query i sees key j iff j <= i + Nk - Nq."""
+    lib = lib or _load()
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    o = np.empty_like(q)
+    lse = np.empty((B, H, Nq), dtype=np.float64)
+    rc = lib.ref_fwd_decode(_p(q), _p(k), _p(v), _p(o), _p(lse), B * H, Nq, Nk, d,
+                            int(bool(causal)), float(scale))
+    if rc == -2:
+        raise ValueError("causal decoding needs Nk >= Nq")
+    if rc:
+        raise MemoryError("oracle: allocation failed")
+    return o, lse

@@ -305,6 +305,43 @@ void ref_dkdv_rows(const double *q, const double *k, const double *v,
     }
 }
 
+/*
+ * Forward with different query and key counts (token-by-token decoding
+ * against a key/value cache: the iplexlaw FlashAttention-2 blog, section
+ * "Document the implementation difference", separates long-prompt
+ * processing from token-by-token generation).  q, o: [BH, Nq, d];
+ * k, v: [BH, Nk, d]; lse: [BH, Nq].  With causal != 0, query i sees key j iff
+ * j <= i + (Nk - Nq): the last query sees every key and the diagonal ends at
+ * the last key, the usual alignment when Nq new tokens extend a cache of
+ * Nk - Nq.  Requires Nk >= Nq when causal (every row then sees >= 1 key).
+ * Returns 0, -1 on allocation failure, -2 on an invalid size.
+ */
+int ref_fwd_decode(const double *q, const double *k, const double *v, double *o,
+                   double *lse, int BH, int Nq, int Nk, int d, int causal,
+                   double scale) {
+    if (causal && Nk < Nq) return -2;
+    const long long rows = (long long)BH * Nq;
+    const int offset = Nk - Nq;
+    int failed = 0;
+#pragma omp parallel reduction(| : failed)
+    {
+        double *p = (double *)malloc(sizeof(double) * (size_t)(Nk > 0 ? Nk : 1));
+        if (!p) failed = 1;
+#pragma omp for schedule(dynamic, 4)
+        for (long long r = 0; r < rows; ++r) {
+            if (!p) continue;
+            const long long bh = r / Nq;
+            const int i = (int)(r % Nq);
+            const int n = causal ? i + offset + 1 : Nk;
+            const size_t kv = (size_t)bh * Nk * d;
+            lse[r] = forward_row(q + (size_t)r * d, k + kv, v + kv, n, d, scale, p,
+                                 o + (size_t)r * d);
+        }
+        free(p);
+    }
+    return failed ? -1 : 0;
+}
+
 /* Threads OpenMP will use (1 without OpenMP). */
 int ref_num_threads(void) {
 #ifdef _OPENMP

@@ -424,6 +424,8 @@ MUTANTS = {
                                 "for (int i = causal ? j + 1 : 0; i < N; ++i)"),
     "rows_dq_drops_D": ("const double ds = p[j] * (dp[j] - Di);\n                for",
                         "const double ds = p[j] * dp[j];\n                for"),
+    "decode_extent_off_by_one": ("const int n = causal ? i + offset + 1 : Nk;",
+                                 "const int n = causal ? i + offset : Nk;"),
 }
 
 
@@ -441,5 +443,82 @@ def test_planted_mistake_is_caught(name, tmp_path):
     lib = oracle.open_library(str(so_path))
     with np.errstate(all="ignore"):
         caught = bool(pin_brute_forward(lib) or pin_numeric_grads(lib)
-                      or pin_library_routine(lib))
+                      or pin_library_routine(lib) or pin_decode(lib))
     assert caught, f"planted mistake {name} passed every pin"
+
+
+# ----------------------------------------------------------------------------
+# decoding: Nq queries against Nk >= Nq keys, causal diagonal ending at the
+# last key
+# ----------------------------------------------------------------------------
+
+def brute_decode(q, k, v, causal, scale, dps=50):
+    """Direct 50-digit summation for Nq queries against Nk keys."""
+    Nq, Nk, d = q.shape[0], k.shape[0], q.shape[1]
+    O, L = [], []
+    with mp.workdps(dps):
+        sc = mp.mpf(float(scale))
+        for i in range(Nq):
+            n = i + Nk - Nq + 1 if causal else Nk
+            w = [mp.exp(sc * mp.fsum(mp.mpf(float(q[i, t])) * mp.mpf(float(k[j, t]))
+                                      for t in range(d))) for j in range(n)]
+            Z = mp.fsum(w)
+            O.append([float(mp.fsum(w[j] * mp.mpf(float(v[j, t])) for j in range(n)) / Z)
+                      for t in range(d)])
+            L.append(float(mp.log(Z)))
+    return np.array(O, dtype=np.float64), np.array(L, dtype=np.float64)
+
+
+def pin_decode(lib=None, tol=1e-13):
+    failures = []
+    for seed, (Nq, Nk, d) in enumerate([(1, 9, 3), (3, 7, 2), (4, 4, 4), (2, 11, 1)]):
+        q, _, _, _ = rng_inputs(300 + seed, 1, 2, Nq, d)
+        _, k, v, _ = rng_inputs(400 + seed, 1, 2, Nk, d)
+        for causal in (False, True):
+            o, lse = oracle.ref_fwd_decode(q, k, v, causal, 0.8, lib=lib)
+            for h in range(2):
+                O, L = brute_decode(q[0, h], k[0, h], v[0, h], causal, 0.8)
+                if not (rel_err(o[0, h], O) <= tol and rel_err(lse[0, h], L) <= tol):
+                    failures.append((Nq, Nk, d, causal, h))
+    return failures
+
+
+def test_decode_brute_force():
+    assert pin_decode() == []
+
+
+def test_decode_library_routine():
+    q, _, _, _ = rng_inputs(500, 2, 3, 5, 16)
+    _, k, v, _ = rng_inputs(501, 2, 3, 77, 16)
+    for causal in (False, True):
+        mask = None
+        if causal:
+            i = np.arange(5)[:, None]
+            j = np.arange(77)[None, :]
+            mask = torch.tensor(j <= i + 77 - 5)
+        to = torch.nn.functional.scaled_dot_product_attention(
+            torch.tensor(q), torch.tensor(k), torch.tensor(v), attn_mask=mask, scale=0.3)
+        o, _ = oracle.ref_fwd_decode(q, k, v, causal, 0.3)
+        assert rel_err(o, to.numpy()) <= 1e-12
+
+
+def test_decode_closed_forms():
+    _, k, v, _ = rng_inputs(502, 1, 2, 30, 6)
+    q = np.zeros((1, 2, 4, 6))
+    o, lse = oracle.ref_fwd_decode(q, k, v, True, 0.5)
+    for i in range(4):            # Q = 0: mean of the visible values
+        n = i + 30 - 4 + 1
+        np.testing.assert_allclose(o[:, :, i], v[:, :, :n].mean(axis=2), atol=1e-14)
+        np.testing.assert_allclose(lse[:, :, i], np.log(n), atol=1e-14)
+    # the last query sees every key, causal or not; Nq == Nk reduces to ref_fwd
+    q, k, v, _ = rng_inputs(503, 1, 2, 12, 5)
+    oc, lc = oracle.ref_fwd_decode(q[:, :, -1:], k, v, True, 0.7)
+    on, ln = oracle.ref_fwd_decode(q[:, :, -1:], k, v, False, 0.7)
+    np.testing.assert_allclose(oc, on, atol=0)
+    for causal in (False, True):
+        a, la = oracle.ref_fwd_decode(q, k, v, causal, 0.7)
+        b, lb = oracle.ref_fwd(q, k, v, causal, 0.7)
+        np.testing.assert_allclose(a, b, atol=0)
+        np.testing.assert_allclose(la, lb, atol=0)
+    with pytest.raises(ValueError):
+        oracle.ref_fwd_decode(q, k[:, :, :5], v[:, :, :5], True, 0.7)
