@@ -146,14 +146,17 @@ struct BwdTraits {
     static constexpr int NBAR = 1 + 2 * NSTAGE + 10 + 2;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
-    static constexpr int NUM_THREADS = 384;  // 3 warpgroups; warps 10-11 idle
-    static constexpr int MMA_WARP = 8;
-    static constexpr int LOAD_WARP = 9;
-    // Register split: P/dS warpgroup grows, dQ drain and MMA/TMA shrink.
-    static constexpr uint32_t REG_COMPUTE = 240;
-    static constexpr uint32_t REG_DRAIN = 120;
-    static constexpr uint32_t REG_CONTROL = 72;
-    static constexpr int REG_BUDGET = 128 * (REG_COMPUTE + REG_DRAIN + REG_CONTROL);
+    // Warps 0-7: two P/dS warpgroups; 8-11: dQ drain; 12: MMA issuer;
+    // 13: TMA producer; 14-15 idle.
+    static constexpr int NUM_THREADS = 512;
+    static constexpr int DRAIN_WARP0 = 8;
+    static constexpr int MMA_WARP = 12;
+    static constexpr int LOAD_WARP = 13;
+    // Register split: P/dS warpgroups grow, dQ drain and MMA/TMA shrink.
+    static constexpr uint32_t REG_COMPUTE = 160;
+    static constexpr uint32_t REG_DRAIN = 96;
+    static constexpr uint32_t REG_CONTROL = 96;
+    static constexpr int REG_BUDGET = 128 * (2 * REG_COMPUTE + REG_DRAIN + REG_CONTROL);
     static constexpr uint32_t TMEM_COLS = 512;
     // TMEM columns: buffer b holds S_b at [128b, 128b+64) (later P | dS) and
     // dP_b at [128b+64, 128b+128) (later the dQ^T of the previous block);
@@ -181,7 +184,7 @@ struct BwdParams {
 };
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1) fa_bwd_main_kernel(
+__global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
     const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
@@ -231,8 +234,8 @@ __global__ void __launch_bounds__(384, 1) fa_bwd_main_kernel(
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sdp_full[b], 1);
-            mbar_init(&sdp_loaded[b], 128);
-            mbar_init(&pds_ready[b], 128);
+            mbar_init(&sdp_loaded[b], 256);
+            mbar_init(&pds_ready[b], 256);
             mbar_init(&dq_full[b], 1);
             mbar_init(&dq_drained[b], 128);
         }
@@ -257,7 +260,7 @@ __global__ void __launch_bounds__(384, 1) fa_bwd_main_kernel(
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const AbortState st{abort_flag, p.err};
-    if (warp >= 8) {
+    if (warp >= T::MMA_WARP) {
       setmaxnreg_dec<T::REG_CONTROL>();
       if (warp == T::LOAD_WARP) {
         // ------------------------------------------------ TMA producer
@@ -329,10 +332,11 @@ __global__ void __launch_bounds__(384, 1) fa_bwd_main_kernel(
 #pragma unroll
                 for (int kk = 0; kk < T::BM / 16; ++kk) {
                     const uint32_t acc = (k > 0 || kk > 0) ? 1u : 0u;
-                    umma_ts(tmem + T::DV_COL, tmem + 128u * b + 8u * kk,
+                    const uint32_t a_col = 128u * b + 32u * (kk >> 1) + 8u * (kk & 1);
+                    umma_ts(tmem + T::DV_COL, tmem + a_col,
                             sdesc_sw128(sq + T::Q_TILE + kk * 2048, T::Q_CHUNK, 1024), T::IDESC_ACC,
                             acc);
-                    umma_ts(tmem + T::DK_COL, tmem + 128u * b + 32u + 8u * kk,
+                    umma_ts(tmem + T::DK_COL, tmem + a_col + 16u,
                             sdesc_sw128(sq + kk * 2048, T::Q_CHUNK, 1024), T::IDESC_ACC, acc);
                 }
             };
@@ -384,10 +388,13 @@ __global__ void __launch_bounds__(384, 1) fa_bwd_main_kernel(
         }
         __syncwarp();
       }
-    } else if (warp < 4) {
+    } else if (warp < T::DRAIN_WARP0) {
         // ------------------------------------------------ P / dS (one thread per key row)
+        // Two warpgroups: warpgroup g handles query columns [32g, 32g+32) of
+        // every key row and rewrites only its own 32 S columns (P, then dS).
         setmaxnreg_inc<T::REG_COMPUTE>();
-        const int lg = warp;
+        const int g = warp >> 2;
+        const int lg = warp & 3;
         const int r = lg * 32 + lane;
         const int kv_row = j * T::BN + r;
         const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
@@ -398,42 +405,49 @@ __global__ void __launch_bounds__(384, 1) fa_bwd_main_kernel(
             ok = __all_sync(0xffffffffu, mbar_wait(&sdp_full[b], (k >> 1) & 1, st));
             if (!ok) break;
             tc_fence_after();
-            uint32_t sv[2][32], dp[2][32];
-            tmem_ld32(tmem + lane_off + 128u * b, sv[0]);
-            tmem_ld32(tmem + lane_off + 128u * b + 32u, sv[1]);
-            tmem_ld32(tmem + lane_off + 128u * b + 64u, dp[0]);
-            tmem_ld32(tmem + lane_off + 128u * b + 96u, dp[1]);
+            const uint32_t s_tm = tmem + lane_off + 128u * b + 32u * g;
+            uint32_t sv[32], dp[32];
+            tmem_ld32(s_tm, sv);
+            tmem_ld32(s_tm + 64u, dp);
             tmem_ld_wait();
             tc_fence_before();
             mbar_arrive(&sdp_loaded[b]);
 
-            const float* lse2 = vec + (k % T::NSTAGE) * 2 * T::BM;
-            const float* dv = lse2 + T::BM;
-            const int qrow0 = (qb0 + k) * T::BM;
-            const int masked = CAUSAL ? kv_row - qrow0 : 0;  // columns c < masked are hidden
-            uint32_t pk[32], dk[32];
+            const float4* l4 = reinterpret_cast<const float4*>(vec + (k % T::NSTAGE) * 2 * T::BM +
+                                                               32 * g);
+            const float4* d4 = l4 + T::BM / 4;
+            const int qrow0 = (qb0 + k) * T::BM + 32 * g;
+            const int masked = CAUSAL ? kv_row - qrow0 : 0;  // columns e < masked are hidden
+            uint32_t pk[16], dk[16];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                float pv[2], dsv[2];
+            for (int e4 = 0; e4 < 8; ++e4) {
+                const float4 lv = l4[e4];
+                const float4 dvv = d4[e4];
+                const float lsv[4] = {lv.x, lv.y, lv.z, lv.w};
+                const float dsv_[4] = {dvv.x, dvv.y, dvv.z, dvv.w};
+                float pr[4], ds[4];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int c = 2 * e + h;
-                    float pr = ex2_approx(fmaf(__uint_as_float(sv[c >> 5][c & 31]), sl2, -lse2[c]));
-                    if (CAUSAL && c < masked) pr = 0.f;
-                    pv[h] = pr;
-                    dsv[h] = pr * (__uint_as_float(dp[c >> 5][c & 31]) - dv[c]);
+                for (int h = 0; h < 4; ++h) {
+                    const int e = 4 * e4 + h;
+                    float x = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -lsv[h]));
+                    if (CAUSAL && e < masked) x = 0.f;
+                    pr[h] = x;
+                    ds[h] = x * (__uint_as_float(dp[e]) - dsv_[h]);
                 }
-                pk[e] = pack_bf16x2(pv[0], pv[1]);
-                dk[e] = pack_bf16x2(dsv[0], dsv[1]);
+                pk[2 * e4] = pack_bf16x2(pr[0], pr[1]);
+                pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
+                dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
+                dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
             }
-            // P^T over S columns [0,32), dS^T over [32,64) (A operands of dV, dK).
-            tmem_st32(tmem + lane_off + 128u * b, pk);
-            tmem_st32(tmem + lane_off + 128u * b + 32u, dk);
-            // dS^T row to shared memory (B operand of dQ^T), 128-byte swizzle.
+            // P^T then dS^T over this warpgroup's own S columns (A operands of
+            // the dV and dK MMAs).
+            tmem_st16(s_tm, pk);
+            tmem_st16(s_tm + 16u, dk);
+            // dS^T half-row to shared memory (B operand of dQ^T), 128-byte swizzle.
             uint8_t* dsrow = smem + T::DS_OFF + (k & 1) * T::DS_TILE;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-                *reinterpret_cast<uint4*>(dsrow + sw128_offset(r, u)) =
+            for (int u = 0; u < 4; ++u)
+                *reinterpret_cast<uint4*>(dsrow + sw128_offset(r, 4 * g + u)) =
                     make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
             fence_proxy_async_smem();
             tmem_st_wait();
@@ -442,53 +456,48 @@ __global__ void __launch_bounds__(384, 1) fa_bwd_main_kernel(
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_done, 0, st));
         if (ok) {
-            // dV and scale*dK -> bf16, staged (128-byte swizzle) in the stage
-            // ring, which no MMA reads any more; TMA-stored 32 rows per warp.
+            // Warpgroup 0 writes dV, warpgroup 1 writes scale*dK: bf16, staged
+            // (128-byte swizzle) in the stage ring, which no MMA reads any
+            // more; TMA-stored 32 rows per warp.
             tc_fence_after();
+            const uint32_t col0 = g ? T::DK_COL : T::DV_COL;
+            const float mul = g ? p.scale : 1.0f;
+            uint8_t* stage = smem + T::ST_OFF + g * T::KV_TILE + lg * 32 * 128;
 #pragma unroll 1
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t col0 = which ? T::DK_COL : T::DV_COL;
-                const float mul = which ? p.scale : 1.0f;
-                uint8_t* stage = smem + T::ST_OFF + which * T::KV_TILE + lg * 32 * 128;
-#pragma unroll 1
-                for (int c = 0; c < D / 32; ++c) {
-                    uint32_t a[32];
-                    tmem_ld32(tmem + lane_off + col0 + 32u * c, a);
-                    tmem_ld_wait();
-                    uint8_t* chunk = stage + (c >> 1) * T::KV_CHUNK;
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t a[32];
+                tmem_ld32(tmem + lane_off + col0 + 32u * c, a);
+                tmem_ld_wait();
+                uint8_t* chunk = stage + (c >> 1) * T::KV_CHUNK;
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        uint4 v;
-                        v.x = pack_bf16x2(__uint_as_float(a[8 * u + 0]) * mul,
-                                          __uint_as_float(a[8 * u + 1]) * mul);
-                        v.y = pack_bf16x2(__uint_as_float(a[8 * u + 2]) * mul,
-                                          __uint_as_float(a[8 * u + 3]) * mul);
-                        v.z = pack_bf16x2(__uint_as_float(a[8 * u + 4]) * mul,
-                                          __uint_as_float(a[8 * u + 5]) * mul);
-                        v.w = pack_bf16x2(__uint_as_float(a[8 * u + 6]) * mul,
-                                          __uint_as_float(a[8 * u + 7]) * mul);
-                        *reinterpret_cast<uint4*>(chunk + sw128_offset(lane, (c & 1) * 4 + u)) = v;
-                    }
+                for (int u = 0; u < 4; ++u) {
+                    uint4 v;
+                    v.x = pack_bf16x2(__uint_as_float(a[8 * u + 0]) * mul,
+                                      __uint_as_float(a[8 * u + 1]) * mul);
+                    v.y = pack_bf16x2(__uint_as_float(a[8 * u + 2]) * mul,
+                                      __uint_as_float(a[8 * u + 3]) * mul);
+                    v.z = pack_bf16x2(__uint_as_float(a[8 * u + 4]) * mul,
+                                      __uint_as_float(a[8 * u + 5]) * mul);
+                    v.w = pack_bf16x2(__uint_as_float(a[8 * u + 6]) * mul,
+                                      __uint_as_float(a[8 * u + 7]) * mul);
+                    *reinterpret_cast<uint4*>(chunk + sw128_offset(lane, (c & 1) * 4 + u)) = v;
                 }
             }
             fence_proxy_async_smem();
             __syncwarp();
             const int wrow0 = j * T::BN + lg * 32;
             if (lane == 0 && wrow0 < N) {
-                for (int c = 0; c < T::CH; ++c) {
-                    uint8_t* base = smem + T::ST_OFF + lg * 32 * 128 + c * T::KV_CHUNK;
-                    tma_store_3d(&tmdV, base, c * 64, wrow0, bh);
-                    tma_store_3d(&tmdK, base + T::KV_TILE, c * 64, wrow0, bh);
-                }
+                for (int c = 0; c < T::CH; ++c)
+                    tma_store_3d(g ? &tmdK : &tmdV, stage + c * T::KV_CHUNK, c * 64, wrow0, bh);
                 bulk_commit_group();
                 bulk_wait_group_read0();
             }
         }
         __syncwarp();
     } else {
-        // ------------------------------------------------ dQ drain (warps 4-7)
+        // ------------------------------------------------ dQ drain (warps 8-11)
         setmaxnreg_dec<T::REG_DRAIN>();
-        const int lg = warp - 4;               // TMEM lanes [32 lg, 32 lg + 32) = head dims
+        const int lg = warp - T::DRAIN_WARP0;  // TMEM lanes [32 lg, 32 lg + 32) = head dims
         const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
         const bool live = lg * 32 < D;         // head dims >= D are padding
         uint8_t* buf = smem + T::DQ_OFF + (live ? lg : 0) * T::DQ_WARP_BYTES;

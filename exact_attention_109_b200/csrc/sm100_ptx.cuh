@@ -76,17 +76,18 @@ __device__ __forceinline__ void raise_abort(const AbortState& st) {
 }
 
 // Waits until the phase with parity `parity` of `bar` has completed.  Returns
-// false -- after flagging the abort -- if that takes longer than kWaitLimitNs,
-// or at once if another role of this CTA has already aborted.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          const AbortState& st) {
+// false -- after flagging the abort -- if that takes longer than `limit_ns`
+// (kWaitLimitNs by default), or at once if another role of this CTA has
+// already aborted.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const AbortState& st,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 31u) == 0u) {
             if (*st.flag) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 raise_abort(st);
                 return false;
             }
