@@ -50,6 +50,20 @@ WORKLOADS = {
                                           dist="row_scaled", seed=5),
 }
 DEFAULT_WORKLOAD = "fwd_bwd_sweep_N8192_d128_causal"
+
+# Decoding (fa_fwd_decode): Nq query rows per sequence against a cache of Nk
+# keys, model width 2048 (H = 16, d = 128); K/V of every workload exceed L2.
+DECODE_WORKLOADS = {
+    "decode_B16_H16_Nq1_Nk8192_d128": dict(B=16, H=16, Nq=1, Nk=8192, d=128, causal=True,
+                                           dist="normal", seed=6),
+    "decode_B1_H16_Nq1_Nk65536_d128": dict(B=1, H=16, Nq=1, Nk=65536, d=128, causal=True,
+                                           dist="normal", seed=6),
+    "decode_B4_H16_Nq4_Nk16384_d128": dict(B=4, H=16, Nq=4, Nk=16384, d=128, causal=True,
+                                           dist="normal", seed=6),
+    "decode_B32_H32_Nq1_Nk4096_d64": dict(B=32, H=32, Nq=1, Nk=4096, d=64, causal=True,
+                                          dist="normal", seed=6),
+}
+DECODE_METRIC = "attention decode (split-KV) HBM GB/s: K/V cache + Q + O bytes per step"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 DATASHEET_BF16_TFLOPS = 2250.0
 
@@ -71,25 +85,29 @@ def load_peaks():
         return dict(FALLBACK_PEAKS, source="fallback")
 
 
-def kernel_sources_hash() -> str:
-    h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "exact_attention_109_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode())
-            h.update(f.read())
-    return h.hexdigest()[:16]
+KERNEL_SOURCES = {
+    "fa_fwd_kernel": "fa_fwd_kernel.cuh",
+    "fa_bwd_main_kernel": "fa_bwd_kernels.cuh",
+    "fa_decode_kernel": "fa_decode_kernel.cuh",
+}
+
+
+def kernel_sources_hash(kernel: str) -> str:
+    """Hash of the source file that holds the kernel's code."""
+    path = os.path.join(ROOT, "exact_attention_109_b200", "csrc", KERNEL_SOURCES[kernel])
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel sources and this workload; otherwise None."""
+    the current source of that kernel and this workload; otherwise None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)
         ent = rec[kernel][workload]
-        if ent.get("sources_hash") != kernel_sources_hash():
+        if ent.get("sources_hash") != kernel_sources_hash(kernel):
             return None
         return float(ent["dram_bytes_per_launch"])
     except Exception:
@@ -381,33 +399,63 @@ def gpu_arm(args, w, wname):
     flops_step = 3.5 * fwd_flops(w)
     value = job_throughput(flops_step, K, world, elapsed_max)
 
-    # ---- end to end through the public API with pinned host buffers
+    # ---- end to end through the public API with pinned host buffers.  Every
+    # step copies its q, k, v, dO in from pinned host memory and its O, LSE,
+    # dQ, dK, dV back out; three streams (host->device, compute,
+    # device->host) and two device buffer sets let step i's copies overlap
+    # the neighbouring steps' compute, as a pipelined caller would run it.
     pin = {x: host[x].pin_memory() for x in ("q", "k", "v", "dO")}
+    outs = ("o", "lse", "dq", "dk", "dv")
     out_host = {x: torch.empty(t_.shape, dtype=t_.dtype, pin_memory=True)
                 for x, t_ in dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv).items()}
     h2d = sum(t_.numel() * t_.element_size() for t_ in pin.values())
     d2h = sum(t_.numel() * t_.element_size() for t_ in out_host.values())
-
-    def e2e_step():
-        for x in ("q", "k", "v", "dO"):
-            dev[x].copy_(pin[x], non_blocking=True)
-        fa.attention_forward(q, k, v, causal, scale, out=o, lse=lse)
-        fa.attention_backward(q, k, v, o, lse, dO, causal, scale, dq=dq, dk=dk, dv=dv,
-                              workspace=ws)
-        for x, t_ in dict(o=o, lse=lse, dq=dq, dk=dk, dv=dv).items():
-            out_host[x].copy_(t_, non_blocking=True)
-
+    bufs = []
     for _ in range(2):
-        e2e_step()
+        bq = {x: torch.empty_like(dev[x]) for x in ("q", "k", "v", "dO")}
+        bo = {"o": torch.empty_like(o), "lse": torch.empty_like(lse),
+              "dq": torch.empty_like(dq), "dk": torch.empty_like(dk), "dv": torch.empty_like(dv)}
+        bufs.append((bq, bo))
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_cmp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
+
+    def e2e_step(i):
+        bq, bo = bufs[i % 2]
+        with torch.cuda.stream(s_in):
+            s_in.wait_event(ev_cmp[i % 2])      # step i-2 has finished reading bq
+            for x in ("q", "k", "v", "dO"):
+                bq[x].copy_(pin[x], non_blocking=True)
+            ev_in[i % 2].record(s_in)
+        with torch.cuda.stream(s_cmp):
+            s_cmp.wait_event(ev_in[i % 2])
+            s_cmp.wait_event(ev_out[i % 2])     # step i-2's results have left bo
+            fa.attention_forward(bq["q"], bq["k"], bq["v"], causal, scale, out=bo["o"],
+                                 lse=bo["lse"], stream=s_cmp)
+            fa.attention_backward(bq["q"], bq["k"], bq["v"], bo["o"], bo["lse"], bq["dO"],
+                                  causal, scale, dq=bo["dq"], dk=bo["dk"], dv=bo["dv"],
+                                  workspace=ws, stream=s_cmp)
+            ev_cmp[i % 2].record(s_cmp)
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(ev_cmp[i % 2])
+            for x in outs:
+                out_host[x].copy_(bo[x], non_blocking=True)
+            ev_out[i % 2].record(s_out)
+
+    for i in range(4):
+        e2e_step(i)
     torch.cuda.synchronize()
-    Ke = max(3, min(K, 20))
+    Ke = max(4, min(K, 20))
     if world > 1:
         dist.barrier()
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(Ke):
-        e2e_step()
-    e1.record(stream)
+    e0.record(s_in)
+    for i in range(Ke):
+        e2e_step(i)
+    s_in.wait_stream(s_out)
+    e1.record(s_in)
     torch.cuda.synchronize()
     e2e_value = job_throughput(flops_step, Ke, world,
                                max_over_ranks(e0.elapsed_time(e1), q.device))
@@ -476,9 +524,213 @@ def gpu_arm(args, w, wname):
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+                "d2h_bytes_per_step": d2h,
+                "note": "public API, pinned host buffers, copies of each step overlap "
+                        "neighbouring steps on separate streams"},
         "gpu_launches": len(stages) * K,
         "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- decoding
+
+
+def decode_bytes(w) -> int:
+    """Algorithmic HBM bytes of one decoding step: every cached key and value
+    row read once, the query rows read, O written (bf16), LSE written (fp32)."""
+    bh = w["B"] * w["H"]
+    return bh * (2 * w["Nk"] * w["d"] * 2 + 2 * w["Nq"] * w["d"] * 2 + w["Nq"] * 4)
+
+
+def decode_config(w, wname):
+    return {"workload": wname, "B": w["B"], "H": w["H"], "Nq": w["Nq"], "Nk": w["Nk"],
+            "d": w["d"], "causal": w["causal"], "inputs": w["dist"], "pass": "decode fwd",
+            "global_batch": w["B"], "seq_len": w["Nk"],
+            "parallelism": "independent head shards per GPU"}
+
+
+def oracle_decode(w, seconds: float):
+    """Time the oracle's decoding reference on whole heads of the workload: as
+    many as fit in about `seconds` (at least one).  Returns (GB/s credited by
+    the same byte count as the GPU line, seconds, heads, cores)."""
+    import oracle
+    from exact_attention_109_b200.inputs import decode_inputs, default_scale, to_f64
+
+    cores = oracle.num_threads()
+    scale = default_scale(w["d"])
+    heads = max(1, min(w["B"] * w["H"], cores))
+    while True:
+        inp = decode_inputs(1, heads, w["Nq"], w["Nk"], w["d"], w["seed"], w["dist"])
+        q, k, v = (to_f64(inp[x]) for x in ("q", "k", "v"))
+        t0 = time.perf_counter()
+        oracle.ref_fwd_decode(q, k, v, w["causal"], scale)
+        t = time.perf_counter() - t0
+        if t * 2 > seconds or heads >= w["B"] * w["H"]:
+            break
+        heads = min(w["B"] * w["H"], heads * 2)
+    return decode_bytes(dict(w, B=1, H=heads)) / t / 1e9, t, heads, cores
+
+
+def decode_reference_arm(args, w, wname):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    per_step = max(0.05, 150.0 / max(1, args.steps + args.warmup))
+    _, _, heads, cores = oracle_decode(w, per_step)
+    import oracle
+    from exact_attention_109_b200.inputs import decode_inputs, default_scale, to_f64
+    inp = decode_inputs(1, heads, w["Nq"], w["Nk"], w["d"], w["seed"], w["dist"])
+    q, k, v = (to_f64(inp[x]) for x in ("q", "k", "v"))
+    scale = default_scale(w["d"])
+    for _ in range(args.warmup):
+        oracle.ref_fwd_decode(q, k, v, w["causal"], scale)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.ref_fwd_decode(q, k, v, w["causal"], scale)
+    total = time.perf_counter() - t0
+    value = decode_bytes(dict(w, B=1, H=heads)) * args.steps / total / 1e9
+    sample = (f"oracle ref_fwd_decode on {heads} of {w['B'] * w['H']} heads per step, "
+              f"credited those heads' bytes")
+    print(json.dumps({
+        "impl": "reference", "metric": DECODE_METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": decode_config(w, wname),
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+    return 0
+
+
+def decode_arm(args, w, wname):
+    import torch
+    import torch.distributed as dist
+
+    import exact_attention_109_b200 as fa
+    from exact_attention_109_b200.inputs import decode_inputs, default_scale
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=torch.device("cuda", local))
+    B, H, Nq, Nk, d, causal = w["B"], w["H"], w["Nq"], w["Nk"], w["d"], w["causal"]
+    scale = default_scale(d)
+    head0, _ = shard_heads(B * H, world, rank)
+    host = decode_inputs(B, H, Nq, Nk, d, w["seed"] + head0, w["dist"])
+    q, k, v = (host[x].cuda() for x in ("q", "k", "v"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    ws_bytes = fa.fa_decode_workspace_size(B, H, Nq, Nk, d)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.current_stream()
+    s = stream.cuda_stream
+    P = [q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr()]
+
+    def step():
+        st = fa.fa_fwd_decode(*P, B, H, Nq, Nk, Nk, d, int(causal), scale,
+                              ws.data_ptr() if ws_bytes else 0, ws_bytes, s)
+        if st != fa.FA_OK:
+            raise fa.FaError(st, "decode step")
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.fa_get_device_error() != fa.FA_OK:
+        raise RuntimeError("decode warm-up: device error")
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    with ClockSampler(local) as clk:
+        time.sleep(0.3)
+        torch.cuda.synchronize()
+        for i in range(K):
+            evs[i].record(stream)
+            step()
+        evs[K].record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if fa.fa_get_device_error() != fa.FA_OK:
+        raise RuntimeError("decode timed region: device error")
+    per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
+    elapsed_max = max_over_ranks(sum(per_step), q.device)
+    nbytes = decode_bytes(w)
+    value = nbytes * K * world / (elapsed_max * 1e-3) / 1e9
+
+    # End to end through the public API: the cache stays resident on the
+    # device (it is the decoding state); each step's query rows come in from
+    # pinned host memory and O, LSE go back out.
+    q_pin = host["q"].pin_memory()
+    o_host = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    l_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    qd = torch.empty_like(q)
+
+    def e2e_step():
+        qd.copy_(q_pin, non_blocking=True)
+        fa.attention_decode(qd, k, v, causal, scale, out=o, lse=lse,
+                            workspace=ws if ws_bytes else None)
+        o_host.copy_(o, non_blocking=True)
+        l_host.copy_(lse, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    Ke = max(4, min(K, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(Ke):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_value = nbytes * Ke * world / (max_over_ranks(e0.elapsed_time(e1), q.device)
+                                       * 1e-3) / 1e9
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks = load_peaks()
+    st, qg, n_splits, chunk = fa.fa_decode_split_plan(
+        B, H, Nq, Nk, d, torch.cuda.get_device_properties(local).multi_processor_count,
+        2 if d == 128 else 3)
+    mean_ms = sum(per_step) / K
+    achieved = nbytes / (mean_ms * 1e-3) / 1e9
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        val, tcpu, heads, cores = oracle_decode(w, 20.0)
+        cpu = {"value": val, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"oracle ref_fwd_decode on {heads} whole heads, {tcpu:.2f} s"}
+    line = {
+        "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": elapsed_max / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 (bf16 inputs)", "data": "synthetic",
+        "config": dict(decode_config(w, wname),
+                       l2=f"no flush: K/V {2 * B * H * Nk * d * 2 / 1e6:.0f} MB > 126 MB L2",
+                       split=f"{n_splits} key splits of {chunk}, {qg} query rows per CTA"),
+        "tokens_per_s": B * Nq * K * world / (elapsed_max * 1e-3),
+        "roofline": {"kernel": "fa_decode_kernel (+ fa_decode_combine_kernel)",
+                     "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "peak_source": f"{peaks['source']} copy bandwidth",
+                     "traffic": recorded_traffic("fa_decode_kernel", wname)},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": q.numel() * 2,
+                "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4,
+                "note": "public API; K/V cache resident on the device, query rows in "
+                        "from pinned host memory, O and LSE back, every step"},
+        "gpu_launches": K * (2 if n_splits > 1 else 1),
+        "clocks": clk.summary(),
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -490,10 +742,16 @@ def main():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS), default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS),
+                    default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.workload in DECODE_WORKLOADS:
+        w = DECODE_WORKLOADS[args.workload]
+        if args.impl == "reference":
+            return decode_reference_arm(args, w, args.workload)
+        return decode_arm(args, w, args.workload)
     w = WORKLOADS[args.workload]
     if args.impl == "reference":
         return reference_arm(args, w, args.workload)

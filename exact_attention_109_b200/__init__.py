@@ -17,6 +17,7 @@ from .api import (  # noqa: F401
     FA_ERR_CUDA, FA_ERR_TIMEOUT, FaError, library, library_path,
     fa_fwd, fa_bwd, fa_bwd_workspace_size, fa_get_device_error, fa_strerror,
     fa_bwd_preprocess, fa_bwd_main, fa_bwd_dq_convert,
-    fa_bwd_noalloc, FA_BWD_NOALLOC_MAX_WORKSPACE_BYTES,
-    attention_forward, attention_backward,
+    fa_bwd_noalloc, FA_BWD_NOALLOC_MAX_WORKSPACE_BYTES, fa_selftest_wait_timeout,
+    fa_fwd_decode, fa_decode_workspace_size, fa_decode_split_plan,
+    attention_forward, attention_backward, attention_decode,
 )

@@ -63,6 +63,16 @@ def library():
     lib.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, f,
                                    vp]
     lib.fa_bwd_noalloc.restype = i
+    ll = ctypes.c_longlong
+    lib.fa_decode_workspace_size.argtypes = [i, i, i, i, i]
+    lib.fa_decode_workspace_size.restype = sz
+    lib.fa_fwd_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, ll, i, i, f, vp, sz, vp]
+    lib.fa_fwd_decode.restype = i
+    ip = ctypes.POINTER(i)
+    lib.fa_decode_split_plan.argtypes = [i, i, i, i, i, i, i, ip, ip, ip]
+    lib.fa_decode_split_plan.restype = i
+    lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
+    lib.fa_selftest_wait_timeout.restype = i
     lib.fa_get_device_error.argtypes = [vp]
     lib.fa_get_device_error.restype = i
     lib.fa_strerror.argtypes = [i]
@@ -136,6 +146,35 @@ def fa_bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
     return int(library().fa_bwd_workspace_size(B, H, N, d))
 
 
+def fa_decode_workspace_size(B: int, H: int, Nq: int, Nk: int, d: int) -> int:
+    return int(library().fa_decode_workspace_size(B, H, Nq, Nk, d))
+
+
+def fa_fwd_decode(q: int, k: int, v: int, o: int, lse: int, B: int, H: int, Nq: int,
+                  Nk: int, kv_rows: int, d: int, causal: int, scale: float,
+                  workspace: int, workspace_bytes: int, stream: int = 0) -> int:
+    """Raw C call with device pointers as integers; returns the status."""
+    return library().fa_fwd_decode(q, k, v, o, lse, B, H, Nq, Nk, int(kv_rows), d,
+                                   int(causal), float(scale), workspace or None,
+                                   int(workspace_bytes), stream or None)
+
+
+def fa_decode_split_plan(B: int, H: int, Nq: int, Nk: int, d: int, sm_count: int,
+                         ctas_per_sm: int):
+    """(status, query rows per CTA, key splits, keys per split) of the host
+    split plan; pure host arithmetic, needs no GPU."""
+    qg, ns, ch = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    st = library().fa_decode_split_plan(B, H, Nq, Nk, d, sm_count, ctas_per_sm,
+                                        ctypes.byref(qg), ctypes.byref(ns),
+                                        ctypes.byref(ch))
+    return st, qg.value, ns.value, ch.value
+
+
+def fa_selftest_wait_timeout(limit_us: int, stream: int = 0) -> int:
+    """Raw C call: enqueue the bounded-wait self-test (see include/fa.h)."""
+    return library().fa_selftest_wait_timeout(int(limit_us), stream or None)
+
+
 def fa_get_device_error(stream: int = 0) -> int:
     return library().fa_get_device_error(stream or None)
 
@@ -202,3 +241,31 @@ def attention_backward(q, k, v, out, lse, dO, causal: bool, scale: float,
                   _ptr(workspace), workspace.numel() * workspace.element_size(),
                   s), "fa_bwd")
     return dq, dk, dv
+
+
+def attention_decode(q, k, v, causal: bool, scale: float, n_keys: int | None = None,
+                     out=None, lse=None, workspace=None, stream=None):
+    """O, LSE = fa_fwd_decode(q, k, v): q [B,H,Nq,d] against the first n_keys
+    rows (default: all) of the cache tensors k, v [B,H,kv_rows,d] (CUDA bf16).
+    With causal, query i sees key j iff j <= i + n_keys - Nq."""
+    B, H, Nq, d = _shape(q)
+    kv_rows = k.shape[2] if k.dim() == 4 else -1
+    Nk = kv_rows if n_keys is None else int(n_keys)
+    _require({"q": q}, (B, H, Nq, d), torch.bfloat16, q.device)
+    _require({"k": k, "v": v}, (B, H, kv_rows, d), torch.bfloat16, q.device)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _require({"out": out}, (B, H, Nq, d), torch.bfloat16, q.device)
+    _require({"lse": lse}, (B, H, Nq), torch.float32, q.device)
+    need = fa_decode_workspace_size(B, H, Nq, Nk, d)
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else 0
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    _check(fa_fwd_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Nq, Nk,
+                         kv_rows, d, int(causal), scale, ws_ptr, ws_bytes, s),
+           "fa_fwd_decode")
+    return out, lse

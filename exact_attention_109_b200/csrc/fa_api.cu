@@ -5,20 +5,44 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
 
 #include "fa.h"
 #include "fa_bwd_kernels.cuh"
+#include "fa_decode_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 
 // Set (bitwise OR) by a kernel whose pipeline wait ran out; one per device.
 __device__ unsigned int g_fa_error_word;
+// Where the wait-timeout self-test kernel reports how its wait ended.
+__device__ int g_fa_probe_result;
 
 namespace {
 
 constexpr int kMaxDevices = 64;
+
+// One CTA waits, through the kernels' bounded wait, on an mbarrier that
+// nothing ever arrives on; the wait runs out after `limit_ns` and records
+// the timeout in the device error word exactly as a stalled pipeline would.
+__global__ void fa_wait_timeout_probe_kernel(unsigned int* err, unsigned long long limit_ns,
+                                             int* completed) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        fa::mbar_init(&bar, 1);
+        abort_flag = 0;
+        fa::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const fa::AbortState st{&abort_flag, err};
+        const bool ok = fa::mbar_wait(&bar, 0, st, limit_ns);
+        *completed = ok ? 1 : 2;
+    }
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
@@ -27,6 +51,8 @@ struct DeviceState {
     std::once_flag once;
     bool ok = false;
     unsigned int* err_word = nullptr;
+    int sm_count = 0;
+    int dec_occ[2][3] = {};  // resident decode CTAs per SM: [d = 64, 128][QG = 1, 2, 4]
 };
 DeviceState g_dev[kMaxDevices];
 
@@ -53,6 +79,25 @@ bool prepare_kernel(K kernel, int bytes, int threads, int reg_budget) {
     cudaFuncAttributes attr{};
     if (cudaFuncGetAttributes(&attr, kernel) != cudaSuccess) return false;
     return attr.numRegs * threads >= reg_budget;
+}
+
+template <int D, int QG>
+bool prepare_decode_one(int* occ) {
+    using T = fa::DecTraits<D>;
+    if (cudaFuncSetAttribute(fa::fa_decode_kernel<D, QG>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             T::SMEM_BYTES) != cudaSuccess)
+        return false;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(occ, fa::fa_decode_kernel<D, QG>,
+                                                         T::THREADS, T::SMEM_BYTES) ==
+               cudaSuccess &&
+           *occ >= 1;
+}
+
+template <int D>
+bool prepare_decode(int (&occ)[3]) {
+    return prepare_decode_one<D, 1>(&occ[0]) && prepare_decode_one<D, 2>(&occ[1]) &&
+           prepare_decode_one<D, 4>(&occ[2]);
 }
 
 // One-time per-device set-up: architecture check, error-word address, and
@@ -87,6 +132,10 @@ fa_status device_setup(int* dev_out, unsigned int** err_out) {
                              fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
         ok &= prepare_kernel(fa::fa_bwd_main_kernel<128, true>, fa::BwdTraits<128>::SMEM_BYTES,
                              fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
+        ok &= cudaDeviceGetAttribute(&s.sm_count, cudaDevAttrMultiProcessorCount, dev) ==
+              cudaSuccess;
+        ok &= prepare_decode<64>(s.dec_occ[0]);
+        ok &= prepare_decode<128>(s.dec_occ[1]);
         s.ok = ok;
     });
     if (!s.ok) {
@@ -341,6 +390,21 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
     return bwd_convert_impl(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
+fa_status fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+    if (limit_us == 0 || limit_us > 2000000u) return FA_ERR_INVALID_ARG;
+    int dev;
+    unsigned int* err;
+    fa_status st = device_setup(&dev, &err);
+    if (st != FA_OK) return st;
+    int* completed = nullptr;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&completed), g_fa_probe_result) !=
+        cudaSuccess)
+        return FA_ERR_CUDA;
+    fa_wait_timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        err, 1000ull * limit_us, completed);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 fa_status fa_get_device_error(void* stream) {
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return FA_ERR_CUDA;
@@ -351,6 +415,183 @@ fa_status fa_get_device_error(void* stream) {
         return FA_ERR_CUDA;
     if (word & fa::kErrTimeout) return FA_ERR_TIMEOUT;
     return word ? FA_ERR_CUDA : FA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ decoding
+
+namespace {
+
+int decode_qgroup_rows(int Nq) { return Nq == 1 ? 1 : Nq == 2 ? 2 : 4; }
+
+long long decode_max_splits(int Nk) {
+    return (static_cast<long long>(Nk) + fa::kDecodeMinChunk - 1) / fa::kDecodeMinChunk;
+}
+
+fa_status decode_check(int B, int H, int Nq, int Nk, int d, float scale) {
+    if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return FA_ERR_INVALID_ARG;
+    if (!(std::isfinite(scale) && scale > 0.f)) return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    const long long bh = static_cast<long long>(B) * H;
+    // Grid indices (one CTA per head x split x query group) are 32-bit.
+    if (bh > (1ll << 24) || Nq > (1 << 24) || Nk > (1 << 30) ||
+        bh * ((Nq + 3) / 4) * decode_max_splits(Nk) > 0x7fffffffll)
+        return FA_ERR_INVALID_ARG;
+    return FA_OK;
+}
+
+// Cost model of the split choice, in units of the time one CTA takes to
+// stream one key row.  One CTA streams at a rate set by the bytes it keeps in
+// flight (its pipeline stages); HBM saturates once about kSatBytesPerSm x SMs
+// bytes are in flight, i.e. with R = that / (bytes per CTA) CTAs streaming.  A
+// wave of n resident CTAs over `chunk` keys therefore lasts
+// chunk * max(1, n / R); each wave adds a fixed ramp (first copies, merge of
+// the warp groups) and splitting adds the merge launch.
+constexpr long long kSatBytesPerSm = 130 << 10;
+constexpr long long kWaveOverheadKeys = 256;
+constexpr long long kMergeOverheadKeys = 128;
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_decode_split_plan(int B, int H, int Nq, int Nk, int d, int sm_count,
+                               int ctas_per_sm, int* qgroup_rows, int* n_splits, int* chunk) {
+    if (!qgroup_rows || !n_splits || !chunk || sm_count < 1 || ctas_per_sm < 1)
+        return FA_ERR_INVALID_ARG;
+    fa_status st = decode_check(B, H, Nq, Nk, d, 1.0f);
+    if (st != FA_OK) return st;
+    constexpr int BK = fa::DecTraits<64>::BK;
+    static_assert(fa::DecTraits<128>::BK == BK, "one key block size for both head dims");
+    const int qg = decode_qgroup_rows(Nq);
+    const long long units = static_cast<long long>(B) * H * ((Nq + qg - 1) / qg);
+    const long long slots = static_cast<long long>(sm_count) * ctas_per_sm;
+    const long long smax = std::min<long long>(decode_max_splits(Nk), 4 * slots);
+    const long long inflight = d == 128
+                                   ? static_cast<long long>(fa::DecTraits<128>::BAR_OFF)
+                                   : static_cast<long long>(fa::DecTraits<64>::BAR_OFF);
+    const double sat = std::max(1.0, static_cast<double>(kSatBytesPerSm) * sm_count / inflight);
+    // The cheapest split count under the cost model above; the smallest on
+    // ties.  Splits that would leave the last one empty are skipped.
+    double best_cost = -1.0;
+    int best_s = 1, best_chunk = (Nk + BK - 1) / BK * BK;
+    for (long long s = 1; s <= smax; ++s) {
+        const long long c = ((Nk + s - 1) / s + BK - 1) / BK * BK;
+        if (s > 1 && c < fa::kDecodeMinChunk) break;
+        const long long s_eff = (Nk + c - 1) / c;
+        if (s_eff != s) continue;
+        const long long ctas = units * s;
+        const long long full_waves = ctas / slots, rest = ctas % slots;
+        double cost = static_cast<double>(full_waves) *
+                      (c * std::max(1.0, slots / sat) + kWaveOverheadKeys);
+        if (rest) cost += c * std::max(1.0, rest / sat) + kWaveOverheadKeys;
+        if (s > 1) cost += kMergeOverheadKeys;
+        if (best_cost < 0 || cost < best_cost * (1.0 - 1e-9)) {
+            best_cost = cost;
+            best_s = static_cast<int>(s);
+            best_chunk = static_cast<int>(c);
+        }
+    }
+    *qgroup_rows = qg;
+    *n_splits = best_s;
+    *chunk = best_chunk;
+    return FA_OK;
+}
+
+size_t fa_decode_workspace_size(int B, int H, int Nq, int Nk, int d) {
+    if (decode_check(B, H, Nq, Nk, d, 1.0f) != FA_OK) return 0;
+    const long long smax = decode_max_splits(Nk);
+    if (smax <= 1) return 0;
+    return static_cast<size_t>(B) * H * Nq * smax * (d + 1) * sizeof(float);
+}
+
+}  // extern "C"
+
+namespace {
+
+template <int D, int QG>
+cudaError_t launch_decode(const fa::DecodeParams& prm, long long bh, cudaStream_t stream) {
+    using T = fa::DecTraits<D>;
+    const long long grid = bh * prm.n_splits * prm.n_qgroups;
+    fa::fa_decode_kernel<D, QG>
+        <<<static_cast<unsigned>(grid), T::THREADS, T::SMEM_BYTES, stream>>>(prm);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || prm.n_splits == 1) return e;
+    const long long rows = bh * prm.Nq;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((rows + 3) / 4));
+    cfg.blockDim = dim3(128);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, fa::fa_decode_combine_kernel<D>,
+                              static_cast<const float*>(prm.part_o),
+                              static_cast<const float*>(prm.part_lse), prm.o, prm.lse, rows,
+                              prm.n_splits);
+}
+
+template <int D>
+cudaError_t launch_decode_d(const fa::DecodeParams& prm, int qg, long long bh,
+                            cudaStream_t stream) {
+    return qg == 1   ? launch_decode<D, 1>(prm, bh, stream)
+           : qg == 2 ? launch_decode<D, 2>(prm, bh, stream)
+                     : launch_decode<D, 4>(prm, bh, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int Nq, int Nk, long long kv_rows, int d, int causal,
+                        float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    fa_status st = decode_check(B, H, Nq, Nk, d, scale);
+    if (st != FA_OK) return st;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (causal && Nk < Nq) return FA_ERR_INVALID_ARG;
+    if (kv_rows < Nk || kv_rows > (1ll << 40)) return FA_ERR_INVALID_ARG;
+    const size_t need = fa_decode_workspace_size(B, H, Nq, Nk, d);
+    if (need > 0 && (!workspace || workspace_bytes < need)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return FA_ERR_MISALIGNED;
+    int dev;
+    unsigned int* err;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    const DeviceState& ds = g_dev[dev];
+    const int qg = decode_qgroup_rows(Nq);
+    const int occ = ds.dec_occ[d == 128][qg == 1 ? 0 : qg == 2 ? 1 : 2];
+    int qg_rows = 0, n_splits = 0, chunk = 0;
+    if ((st = fa_decode_split_plan(B, H, Nq, Nk, d, ds.sm_count, occ, &qg_rows, &n_splits,
+                                   &chunk)) != FA_OK)
+        return st;
+    const long long bh = static_cast<long long>(B) * H;
+    fa::DecodeParams prm;
+    prm.q = static_cast<const __nv_bfloat16*>(q);
+    prm.k = static_cast<const __nv_bfloat16*>(k);
+    prm.v = static_cast<const __nv_bfloat16*>(v);
+    prm.o = static_cast<__nv_bfloat16*>(o);
+    prm.lse = lse;
+    prm.part_o = static_cast<float*>(workspace);
+    prm.part_lse = n_splits > 1 ? prm.part_o + bh * Nq * n_splits * d : nullptr;
+    prm.err = err;
+    prm.kv_rows = kv_rows;
+    prm.Nq = Nq;
+    prm.Nk = Nk;
+    prm.n_qgroups = (Nq + qg - 1) / qg;
+    prm.n_splits = n_splits;
+    prm.chunk = chunk;
+    prm.causal = causal;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = d == 64 ? launch_decode_d<64>(prm, qg, bh, s)
+                                  : launch_decode_d<128>(prm, qg, bh, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 }  // extern "C"

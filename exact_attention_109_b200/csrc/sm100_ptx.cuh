@@ -116,6 +116,18 @@ __device__ __forceinline__ void setmaxnreg_dec() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(R));
 }
 
+// Programmatic dependent launch: a grid launched with programmatic stream
+// serialization may start before its predecessor on the stream ends;
+// grid_dependency_wait() returns once the predecessor has completed and its
+// memory operations are visible.  grid_launch_dependents() lets the
+// dependent grid be scheduled before this one ends.
+__device__ __forceinline__ void grid_dependency_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Named barrier over `nthreads` threads (multiple of 32), id in [1, 15].
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");

@@ -53,6 +53,24 @@ def attention_inputs(B: int, H: int, N: int, d: int, seed: int,
     return out
 
 
+def decode_inputs(B: int, H: int, Nq: int, Nk: int, d: int, seed: int,
+                  dist: str = "normal"):
+    """CPU bf16 q [B,H,Nq,d] and k, v [B,H,Nk,d] for decoding (Nq query rows
+    against Nk cached keys); same recipe and draw order (q, k, v) as above."""
+    gen = torch.Generator("cpu").manual_seed(int(seed))
+    out = {}
+    for name, n in (("q", Nq), ("k", Nk), ("v", Nk)):
+        shape = (B, H, n, d)
+        if dist == "normal":
+            x = _normal(gen, shape)
+        elif dist == "row_scaled":
+            x = _row_scaled(gen, shape)
+        else:
+            raise ValueError(f"unknown input distribution {dist!r}")
+        out[name] = x.to(torch.bfloat16)
+    return out
+
+
 def default_scale(d: int) -> float:
     """1/sqrt(d) rounded to fp32, the value both sides receive."""
     return float(np.float32(1.0 / math.sqrt(d)))

@@ -164,12 +164,71 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
                          int d, int causal, float scale, void* stream);
 
 /*
+ * Decoding: N_q query rows against N_k >= N_q cached keys, N_q small.
+ * iplexlaw blog "FlashAttention-2 GPU work partitioning", section "What the
+ * paper measures": prefill and token-by-token decoding have different
+ * bottlenecks and are measured apart.  Decoding reads every cached key and
+ * value once for a few query rows, so it is bound by HBM bandwidth; the key
+ * range is split across CTAs ("split-KV") and the partial results merged
+ * with the log-sum-exp rule of the online softmax ("Tiling preserves the
+ * attention calculation").
+ *
+ * fa_fwd_decode -- O = softmax(scale * Q K^T [+ causal mask]) V for
+ *   q        [B,H,Nq,d] bf16, read only.
+ *   k, v     [B,H,kv_rows,d] bf16, read only; the first Nk rows of every
+ *            head are the keys (a cache allocated for kv_rows >= Nk rows).
+ *   o        [B,H,Nq,d] bf16, written.
+ *   lse      [B,H,Nq] fp32, written: natural-log LSE over the visible keys.
+ *   causal   0 or 1.  The query rows are the LAST Nq positions of the
+ *            sequence: query i (0-based) sees key j iff j <= i + Nk - Nq
+ *            (needs Nk >= Nq); for Nq = Nk this is fa_fwd's mask.
+ *   workspace  device buffer of >= fa_decode_workspace_size(B,H,Nq,Nk,d)
+ *            bytes, 256-byte aligned, clobbered; may be NULL when that size
+ *            is 0 (Nk <= 256).
+ * Arithmetic: fp32 scores, weights and accumulation from the bf16 inputs.
+ * Intended for Nq <= 16 (query rows are handled four at a time, and every
+ * group of four re-reads the keys, mostly from L2); any Nq >= 1 is correct.
+ * One launch, plus a merge launch when the keys were split.
+ * Errors: as fa_fwd; FA_ERR_INVALID_ARG also for kv_rows < Nk, causal with
+ * Nk < Nq, or a missing / too small workspace.
+ */
+size_t fa_decode_workspace_size(int B, int H, int Nq, int Nk, int d);
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o,
+                        float* lse, int B, int H, int Nq, int Nk,
+                        long long kv_rows, int d, int causal, float scale,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fa_decode_split_plan -- the work split fa_fwd_decode uses on a GPU with
+ * `sm_count` SMs that holds `ctas_per_sm` decode CTAs each: query rows per
+ * CTA (1, 2 or 4), the number of key splits per head, and the keys per split
+ * (a multiple of 64, at least 256 when the keys are split).  Host
+ * arithmetic only; touches no GPU.  Errors: FA_ERR_INVALID_ARG /
+ * FA_ERR_UNSUPPORTED for sizes fa_fwd_decode would reject.
+ */
+fa_status fa_decode_split_plan(int B, int H, int Nq, int Nk, int d,
+                               int sm_count, int ctas_per_sm,
+                               int* qgroup_rows, int* n_splits, int* chunk);
+
+/*
  * fa_get_device_error -- synchronises `stream`, then reads and clears the
  * current device's error word.  Returns FA_ERR_TIMEOUT if a kernel's bounded
  * pipeline wait ran out since the last call, FA_ERR_CUDA if the stream
  * reports a CUDA error, FA_OK otherwise.
  */
 fa_status fa_get_device_error(void* stream);
+
+/*
+ * fa_selftest_wait_timeout -- exercises the failure path of the bounded
+ * device waits without faulting or hanging the GPU: enqueues one tiny kernel
+ * whose single wait, on an mbarrier that nothing arrives on, runs out after
+ * `limit_us` microseconds (1 .. 2,000,000) and records FA_ERR_TIMEOUT in the
+ * device error word, exactly as a stalled attention pipeline would.  The
+ * following fa_get_device_error(stream) returns FA_ERR_TIMEOUT (and clears
+ * the word); the context stays usable.  Errors: FA_ERR_INVALID_ARG for a
+ * limit out of range, FA_ERR_UNSUPPORTED / FA_ERR_CUDA as for fa_fwd.
+ */
+fa_status fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
 
 /* fa_strerror -- static, human-readable name of a status. */
 const char* fa_strerror(fa_status status);
