@@ -48,6 +48,17 @@ WORKLOADS = {
                                           dist="row_scaled", seed=4),
     "gpt_layer_b_B2_N8192_H20_d128": dict(B=2, H=20, N=8192, d=128, causal=True,
                                           dist="row_scaled", seed=5),
+    "long_B1_H16_N65536_d128_causal": dict(B=1, H=16, N=65536, d=128, causal=True,
+                                           dist="normal", seed=3),
+}
+
+# Sequence-sharded (ring) attention, G virtual ranks on one GPU: the long
+# single-sequence shape split into G shards of N/G tokens.
+RING_WORKLOADS = {
+    "ring_G4_B1_H16_N65536_d128_causal": dict(B=1, H=16, N=65536, d=128, causal=True,
+                                              dist="normal", seed=3, G=4),
+    "ring_G2_B2_H16_N8192_d128_causal": dict(B=2, H=16, N=8192, d=128, causal=True,
+                                             dist="normal", seed=2, G=2),
 }
 DEFAULT_WORKLOAD = "fwd_bwd_sweep_N8192_d128_causal"
 
@@ -736,17 +747,132 @@ def decode_arm(args, w, wname):
     return 0
 
 
+# ---------------------------------------------------------------- ring
+
+
+def ring_arm(args, w, wname):
+    """G virtual ranks on this GPU (exact_attention_109_b200.ring.run_local):
+    one step = the ring forward and backward over the whole sequence, every
+    (query shard, key shard) pair through the CUDA kernels, every rotation a
+    device copy of the bytes a ring would move."""
+    import torch
+
+    import exact_attention_109_b200 as fa
+    from exact_attention_109_b200 import ring
+    from exact_attention_109_b200.inputs import attention_inputs, default_scale
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        print(json.dumps({"metric": METRIC, "error": "ring workloads run G virtual ranks on "
+                          "one GPU; across GPUs the ring runs through ring.run_nccl"}))
+        return 1
+    torch.cuda.set_device(0)
+    B, H, N, d, causal, G = w["B"], w["H"], w["N"], w["d"], w["causal"], w["G"]
+    scale = default_scale(d)
+    host = attention_inputs(B, H, N, d, w["seed"], w["dist"], with_dout=True)
+    q, k, v, dO = (host[x].cuda() for x in ("q", "k", "v", "dO"))
+    stream = torch.cuda.current_stream()
+
+    def step():
+        return ring.local_ring_attention(q, k, v, dO, causal, scale, G)
+
+    def plain_step():
+        o, lse = fa.attention_forward(q, k, v, causal, scale)
+        fa.attention_backward(q, k, v, o, lse, dO, causal, scale)
+
+    for _ in range(args.warmup):
+        step()
+        plain_step()
+    torch.cuda.synchronize()
+    if fa.fa_get_device_error() != fa.FA_OK:
+        raise RuntimeError("ring warm-up: device error")
+    K = args.steps
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    with ClockSampler(0) as clk:
+        time.sleep(0.3)
+        torch.cuda.synchronize()
+        for i in range(K):
+            ev[i].record(stream)
+            step()
+        ev[K].record(stream)
+        torch.cuda.synchronize()
+    ring_ms = ev[0].elapsed_time(ev[K]) / K
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K):
+        plain_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    plain_ms = e0.elapsed_time(e1) / K
+    if fa.fa_get_device_error() != fa.FA_OK:
+        raise RuntimeError("ring timed region: device error")
+    flops = 3.5 * fwd_flops(w)
+    value = flops / (ring_ms * 1e-3) / 1e12
+
+    # end to end: q, k, v, dO in from pinned host memory, O, LSE, dQ, dK, dV out
+    pin = {x: host[x].pin_memory() for x in ("q", "k", "v", "dO")}
+    dev = {x: torch.empty_like(q) for x in pin}
+    outs = None
+    Ke = max(2, min(K, 5))
+    e0.record(stream)
+    for _ in range(Ke):
+        for x in pin:
+            dev[x].copy_(pin[x], non_blocking=True)
+        got = ring.local_ring_attention(dev["q"], dev["k"], dev["v"], dev["dO"], causal, scale, G)
+        outs = [t.to("cpu", non_blocking=True) for t in got]
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e = flops / (e0.elapsed_time(e1) / Ke * 1e-3) / 1e12
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    peaks = load_peaks()
+    cpu = None
+    if not args.no_cpu_baseline:
+        run, R, cores, credit = oracle_sample(w, 20.0)
+        t = run(R)
+        cpu = {"value": credit(R) / t / 1e12, "unit": "TFLOP/s", "cores": cores,
+               "kind": "oracle",
+               "sample": f"{R} of {N} query rows and key rows of one head (whole-sequence "
+                         f"fwd+bwd outputs), credited {R}/{N} of the head's FLOPs"}
+    achieved = value
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ring_ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w, wname), **{
+            "G": G, "pass": "ring fwd+bwd",
+            "parallelism": f"ring of {G} virtual ranks on one GPU",
+            "l2": f"no flush: per-step working set {9 * B * H * N * d * 2 / 1e6:.0f} MB"}),
+        "plain_fwd_bwd_tflops": flops / (plain_ms * 1e-3) / 1e12,
+        "ring_overhead": ring_ms / plain_ms - 1.0,
+        "roofline": {"kernel": "whole ring step (fa_fwd, fa_lse_merge, fa_bwd_*)",
+                     "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "peak_source": f"{peaks['source']} (burst)", "traffic": None},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "note": "public API, serial copies"},
+        "gpu_launches": None,
+        "clocks": clk.summary()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS),
+    ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS)
+                    + sorted(RING_WORKLOADS),
                     default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.workload in RING_WORKLOADS:
+        if args.impl == "reference":
+            return reference_arm(args, RING_WORKLOADS[args.workload], args.workload)
+        return ring_arm(args, RING_WORKLOADS[args.workload], args.workload)
     if args.workload in DECODE_WORKLOADS:
         w = DECODE_WORKLOADS[args.workload]
         if args.impl == "reference":

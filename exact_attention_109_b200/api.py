@@ -71,6 +71,13 @@ def library():
     ip = ctypes.POINTER(i)
     lib.fa_decode_split_plan.argtypes = [i, i, i, i, i, i, i, ip, ip, ip]
     lib.fa_decode_split_plan.restype = i
+    lib.fa_lse_merge.argtypes = [vp, vp, vp, vp, vp, ll, i, i, vp]
+    lib.fa_lse_merge.restype = i
+    lib.fa_bwd_main_accumulate.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, sz,
+                                           vp]
+    lib.fa_bwd_main_accumulate.restype = i
+    lib.fa_convert_f32_bf16.argtypes = [vp, vp, ll, vp]
+    lib.fa_convert_f32_bf16.restype = i
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
     lib.fa_selftest_wait_timeout.restype = i
     lib.fa_get_device_error.argtypes = [vp]
@@ -168,6 +175,26 @@ def fa_decode_split_plan(B: int, H: int, Nq: int, Nk: int, d: int, sm_count: int
                                         ctypes.byref(qg), ctypes.byref(ns),
                                         ctypes.byref(ch))
     return st, qg.value, ns.value, ch.value
+
+
+def fa_lse_merge(o_acc: int, lse_acc: int, o_part: int, lse_part: int, o_out: int,
+                 rows: int, d: int, init: int, stream: int = 0) -> int:
+    """Raw C call: fold a partial (O, LSE) into a running fp32 one."""
+    return library().fa_lse_merge(o_acc, lse_acc, o_part, lse_part, o_out or None, int(rows),
+                                  d, int(init), stream or None)
+
+
+def fa_bwd_main_accumulate(q: int, k: int, v: int, dO: int, dk_acc: int, dv_acc: int, B: int,
+                           H: int, N: int, d: int, causal: int, scale: float, workspace: int,
+                           workspace_bytes: int, stream: int = 0) -> int:
+    """Raw C call: fa_bwd_main adding dK, dV into fp32 accumulators."""
+    return library().fa_bwd_main_accumulate(q, k, v, dO, dk_acc, dv_acc, B, H, N, d,
+                                            int(causal), float(scale), workspace,
+                                            int(workspace_bytes), stream or None)
+
+
+def fa_convert_f32_bf16(src: int, dst: int, n: int, stream: int = 0) -> int:
+    return library().fa_convert_f32_bf16(src, dst, int(n), stream or None)
 
 
 def fa_selftest_wait_timeout(limit_us: int, stream: int = 0) -> int:

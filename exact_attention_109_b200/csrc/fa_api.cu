@@ -14,6 +14,7 @@
 #include "fa_bwd_kernels.cuh"
 #include "fa_decode_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
+#include "fa_merge_kernels.cuh"
 
 // Set (bitwise OR) by a kernel whose pipeline wait ran out; one per device.
 __device__ unsigned int g_fa_error_word;
@@ -341,9 +342,96 @@ fa_status bwd_convert_impl(void* dq, int B, int H, int N, int d, float scale, vo
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+fa_status bwd_accum_impl(const void* q, const void* k, const void* v, const void* dO,
+                         float* dk_acc, float* dv_acc, int B, int H, int N, int d, int causal,
+                         float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !dO || !dk_acc || !dv_acc) return FA_ERR_INVALID_ARG;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    fa::BwdWorkspace ws;
+    int dev;
+    unsigned int* err;
+    fa_status st = bwd_common(B, H, N, d, scale, workspace, workspace_bytes, &ws, &dev, &err);
+    if (st != FA_OK) return st;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(dO) || !aligned16(dk_acc) ||
+        !aligned16(dv_acc))
+        return FA_ERR_MISALIGNED;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    if (!load_encode()) return FA_ERR_CUDA;
+    const long long bh = static_cast<long long>(B) * H;
+    CUtensorMap mq, mk, mv, mdo, mdk, mdv, macc;
+    if (!encode_bf16(&mq, q, d, N, bh, fa::kBwdBM) || !encode_bf16(&mk, k, d, N, bh, 128) ||
+        !encode_bf16(&mv, v, d, N, bh, 128) || !encode_bf16(&mdo, dO, d, N, bh, fa::kBwdBM) ||
+        !encode_3d(&mdk, dk_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, 32) ||
+        !encode_3d(&mdv, dv_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, N, bh, 32, 32) ||
+        !encode_3d(&macc, ws.dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, d, ws.n_pad, bh, 32,
+                   fa::kBwdBM))
+        return FA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int ibh = static_cast<int>(bh);
+    cudaError_t e;
+    if (d == 64)
+        e = causal ? fa::launch_bwd_main<64, true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                   macc, err, s, 1)
+                   : fa::launch_bwd_main<64, false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                    macc, err, s, 1);
+    else
+        e = causal ? fa::launch_bwd_main<128, true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                    macc, err, s, 1)
+                   : fa::launch_bwd_main<128, false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk,
+                                                     mdv, macc, err, s, 1);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
+
+fa_status fa_bwd_main_accumulate(const void* q, const void* k, const void* v, const void* dO,
+                                 float* dk_acc, float* dv_acc, int B, int H, int N, int d,
+                                 int causal, float scale, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    return bwd_accum_impl(q, k, v, dO, dk_acc, dv_acc, B, H, N, d, causal, scale, workspace,
+                          workspace_bytes, stream);
+}
+
+fa_status fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                       void* o_out, long long rows, int d, int init, void* stream) {
+    if (!o_acc || !lse_acc || !o_part || !lse_part || rows < 1 || (init != 0 && init != 1))
+        return FA_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+    if (rows > (1ll << 40)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(o_acc) || !aligned16(o_part) || !aligned16(o_out)) return FA_ERR_MISALIGNED;
+    int dev;
+    unsigned int* err;
+    fa_status st = device_setup(&dev, &err);
+    if (st != FA_OK) return st;
+    const long long threads = rows * (d / 8);
+    const unsigned grid = static_cast<unsigned>((threads + 255) / 256);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const auto* op = static_cast<const __nv_bfloat16*>(o_part);
+    auto* oo = static_cast<__nv_bfloat16*>(o_out);
+    if (d == 64)
+        fa::fa_lse_merge_kernel<64><<<grid, 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo, rows,
+                                                         init);
+    else
+        fa::fa_lse_merge_kernel<128><<<grid, 256, 0, s>>>(o_acc, lse_acc, op, lse_part, oo, rows,
+                                                          init);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_convert_f32_bf16(const float* src, void* dst, long long n, void* stream) {
+    if (!src || !dst || n < 8 || n % 8 != 0 || n > (1ll << 42)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(src) || !aligned16(dst)) return FA_ERR_MISALIGNED;
+    int dev;
+    unsigned int* err;
+    fa_status st = device_setup(&dev, &err);
+    if (st != FA_OK) return st;
+    const long long n8 = n / 8;
+    fa::fa_f32_to_bf16_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0,
+                                 static_cast<cudaStream_t>(stream)>>>(
+        src, static_cast<__nv_bfloat16*>(dst), n8);
+    return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
 
 fa_status fa_bwd_preprocess(const void* o, const float* lse, const void* dO, int B, int H, int N,
                             int d, void* workspace, size_t workspace_bytes, void* stream) {

@@ -168,6 +168,7 @@ struct BwdTraits {
     static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, BM, 1, 1);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(2 * KV_TILE <= NSTAGE * STAGE_BYTES, "dK/dV staging fits the stage ring");
+    static_assert(8 * 2 * 4096 <= NSTAGE * STAGE_BYTES, "fp32 dK/dV boxes fit the stage ring");
 };
 
 struct BwdParams {
@@ -179,6 +180,7 @@ struct BwdParams {
     int bh_count;
     int n_kv;        // ceil(N / 128)
     int n_q;         // ceil(N / 64)
+    int accum;       // 0: write bf16 dK, dV; 1: add them to fp32 accumulators
     float scale;
     float scale_log2;
 };
@@ -455,7 +457,42 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
             mbar_arrive(&pds_ready[b]);
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_done, 0, st));
-        if (ok) {
+        if (ok && p.accum) {
+            // Accumulating: warpgroup 0 adds dV, warpgroup 1 adds scale*dK
+            // to fp32 [B*H][N][D] buffers with TMA bulk reduce-adds of
+            // [32 rows][32 head dims] boxes (128-byte swizzle), staged two
+            // boxes per warp in the stage ring, which no MMA reads any more.
+            tc_fence_after();
+            const uint32_t col0 = g ? T::DK_COL : T::DV_COL;
+            const float mul = g ? p.scale : 1.0f;
+            uint8_t* stage = smem + T::ST_OFF + (g * 4 + lg) * 2 * 4096;
+            const int wrow0 = j * T::BN + lg * 32;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t a[32];
+                tmem_ld32(tmem + lane_off + col0 + 32u * c, a);
+                tmem_ld_wait();
+                uint8_t* box = stage + (c & 1) * 4096;
+                if (c >= 2) {
+                    if (lane == 0) bulk_wait_group_read<1>();  // box c-2 was read
+                    __syncwarp();
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u)
+                    *reinterpret_cast<float4*>(box + sw128_offset(lane, u)) =
+                        make_float4(__uint_as_float(a[4 * u + 0]) * mul,
+                                    __uint_as_float(a[4 * u + 1]) * mul,
+                                    __uint_as_float(a[4 * u + 2]) * mul,
+                                    __uint_as_float(a[4 * u + 3]) * mul);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0 && wrow0 < N) {
+                    tma_reduce_add_3d(g ? &tmdK : &tmdV, box, 32 * c, wrow0, bh);
+                    bulk_commit_group();
+                }
+            }
+            if (lane == 0 && wrow0 < N) bulk_wait_group0();
+        } else if (ok) {
             // Warpgroup 0 writes dV, warpgroup 1 writes scale*dK: bf16, staged
             // (128-byte swizzle) in the stage ring, which no MMA reads any
             // more; TMA-stored 32 rows per warp.
@@ -561,7 +598,7 @@ cudaError_t launch_bwd_main(int bh, int N, float scale, const BwdWorkspace& ws,
                             const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const CUtensorMap& mdo, const CUtensorMap& mdk,
                             const CUtensorMap& mdv, const CUtensorMap& macc, unsigned int* err,
-                            cudaStream_t s) {
+                            cudaStream_t s, int accum = 0) {
     using T = BwdTraits<D>;
     BwdParams prm;
     prm.lse2 = ws.lse2;
@@ -572,6 +609,7 @@ cudaError_t launch_bwd_main(int bh, int N, float scale, const BwdWorkspace& ws,
     prm.bh_count = bh;
     prm.n_kv = (N + T::BN - 1) / T::BN;
     prm.n_q = (N + T::BM - 1) / T::BM;
+    prm.accum = accum;
     prm.scale = scale;
     prm.scale_log2 = scale * 1.4426950408889634f;
     const long long grid = static_cast<long long>(bh) * prm.n_kv;

@@ -1,0 +1,259 @@
+"""Sequence-sharded attention across devices (Ring Attention).
+
+Ring Attention with Blockwise Transformers (abstract): the sequence is spread
+over a ring of devices; each device keeps its block of queries while the
+key/value blocks travel around the ring, the transfer of the next block
+overlapping the blockwise attention on the current one, so the context length
+grows with the number of devices.  Every (query shard, key/value shard) pair
+is an ordinary attention problem of the shard length, computed by the CUDA
+library (``fa_fwd`` / ``fa_bwd_main_accumulate``); the pairs' results are
+folded together with the log-sum-exp rule (``fa_lse_merge``).
+
+Layout: rank r of a ring of G holds positions [r n, (r+1) n) of a sequence of
+G n tokens: q, k, v, dO, O as [B, H, n, d] bf16, LSE as [B, H, n] fp32.
+Causal masking is by global position, so for query shard r the key shards
+j < r are fully visible, shard r is causal, and shards j > r are skipped.
+
+Each rank's schedule is written once, as a generator (``forward_program`` /
+``backward_program``) that yields at its exchange points:
+``("start", sends, recvs)`` posts one step of the rotation -- every tensor in
+``sends`` goes to the next rank, every tensor in ``recvs`` is filled from the
+previous rank -- and ``("wait",)`` waits for everything posted.  Two runners
+drive it: ``run_nccl`` with torch.distributed point-to-point operations (one
+process per GPU; over NVLink / NVSwitch with NCCL), and ``run_local``, which
+runs G virtual ranks in lockstep in one process and performs each rotation
+as device-to-device copies (the same bytes a ring would move), for checking
+the whole scheme on one GPU.
+
+The forward sends key/value blocks before computing on the current ones, so
+transfer and compute overlap.  In the backward the dK/dV accumulators travel
+with their key/value block and are sent after the block's gradient is added;
+after G rotations every rank holds its own shard's accumulators again.
+
+This module only marshals buffers and orders calls; all arithmetic runs in
+the CUDA library (an ``ops`` object may be substituted to exercise the
+schedule on CPU in tests).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import api as _api
+
+
+# ---------------------------------------------------------------- compute ops
+
+
+class CudaOps:
+    """The per-step arithmetic, through the library's C ABI."""
+
+    def fwd(self, q, k, v, causal, scale):
+        return _api.attention_forward(q, k, v, causal, scale)
+
+    def merge(self, o_acc, lse_acc, o_part, lse_part, o_out, init):
+        rows = lse_acc.numel()
+        st = _api.fa_lse_merge(o_acc.data_ptr(), lse_acc.data_ptr(), o_part.data_ptr(),
+                               lse_part.data_ptr(), o_out.data_ptr() if o_out is not None else 0,
+                               rows, o_acc.shape[-1], int(init),
+                               torch.cuda.current_stream(o_acc.device).cuda_stream)
+        _api._check(st, "fa_lse_merge")
+
+    def bwd_prepare(self, o, lse, dO):
+        B, H, n, d = o.shape
+        nbytes = _api.fa_bwd_workspace_size(B, H, n, d)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=o.device)
+        st = _api.fa_bwd_preprocess(o.data_ptr(), lse.data_ptr(), dO.data_ptr(), B, H, n, d,
+                                    ws.data_ptr(), nbytes,
+                                    torch.cuda.current_stream(o.device).cuda_stream)
+        _api._check(st, "fa_bwd_preprocess")
+        return ws
+
+    def bwd_accumulate(self, ws, q, k, v, dO, dk_acc, dv_acc, causal, scale):
+        B, H, n, d = q.shape
+        st = _api.fa_bwd_main_accumulate(q.data_ptr(), k.data_ptr(), v.data_ptr(), dO.data_ptr(),
+                                         dk_acc.data_ptr(), dv_acc.data_ptr(), B, H, n, d,
+                                         int(causal), scale, ws.data_ptr(), ws.numel(),
+                                         torch.cuda.current_stream(q.device).cuda_stream)
+        _api._check(st, "fa_bwd_main_accumulate")
+
+    def bwd_finish(self, ws, q, scale):
+        B, H, n, d = q.shape
+        dq = torch.empty_like(q)
+        st = _api.fa_bwd_dq_convert(dq.data_ptr(), B, H, n, d, scale, ws.data_ptr(), ws.numel(),
+                                    torch.cuda.current_stream(q.device).cuda_stream)
+        _api._check(st, "fa_bwd_dq_convert")
+        return dq
+
+    def to_bf16(self, x):
+        out = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+        st = _api.fa_convert_f32_bf16(x.data_ptr(), out.data_ptr(), x.numel(),
+                                      torch.cuda.current_stream(x.device).cuda_stream)
+        _api._check(st, "fa_convert_f32_bf16")
+        return out
+
+
+# ---------------------------------------------------------------- schedules
+
+
+def _visible(causal: bool, rank: int, shard: int) -> bool:
+    return (not causal) or shard <= rank
+
+
+def _last_visible_step(causal: bool, rank: int, world: int) -> int:
+    # step s holds key shard (rank - s) mod world; causal ranks see s = 0..rank
+    return rank if causal else world - 1
+
+
+def forward_program(q, k, v, causal: bool, scale: float, rank: int, world: int, ops=None):
+    """Rank `rank`'s forward: returns (O bf16, LSE fp32) of its query shard."""
+    ops = ops or CudaOps()
+    B, H, n, d = q.shape
+    o_acc = torch.empty((B, H, n, d), dtype=torch.float32, device=q.device)
+    lse_acc = torch.empty((B, H, n), dtype=torch.float32, device=q.device)
+    o_out = torch.empty_like(q)
+    # The caller's k, v are only ever sent; received blocks alternate between
+    # two buffers of our own (one while only two ranks rotate).
+    bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(2, world - 1))]
+    cur = (k, v)
+    last = _last_visible_step(causal, rank, world)
+    first = True
+    for s in range(world):
+        shard = (rank - s) % world
+        if s < world - 1:
+            nxt = bufs[s % 2]
+            yield ("start", list(cur), list(nxt))
+        if _visible(causal, rank, shard):
+            o_p, l_p = ops.fwd(q, cur[0], cur[1], causal and shard == rank, scale)
+            ops.merge(o_acc, lse_acc, o_p, l_p, o_out if s == last else None, first)
+            first = False
+        if s < world - 1:
+            yield ("wait",)
+            cur = nxt
+    return o_out, lse_acc
+
+
+def backward_program(q, k, v, o, lse, dO, causal: bool, scale: float, rank: int, world: int,
+                     ops=None):
+    """Rank `rank`'s backward: returns (dQ, dK, dV) bf16 of its shards, given
+    its query shard's final O and LSE (from forward_program)."""
+    ops = ops or CudaOps()
+    ws = ops.bwd_prepare(o, lse, dO)
+    dk_acc = torch.zeros(k.shape, dtype=torch.float32, device=k.device)
+    dv_acc = torch.zeros(v.shape, dtype=torch.float32, device=v.device)
+    bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(2, world - 1))]
+    kv = (k, v)  # the caller's k, v are only sent, as in the forward
+    acc = (dk_acc, dv_acc)
+    acc_n = (torch.empty_like(dk_acc), torch.empty_like(dv_acc)) if world > 1 else None
+    for s in range(world):
+        shard = (rank - s) % world
+        if s < world - 1:
+            kv_n = bufs[s % 2]
+            yield ("start", list(kv), list(kv_n))
+        if _visible(causal, rank, shard):
+            ops.bwd_accumulate(ws, q, kv[0], kv[1], dO, acc[0], acc[1],
+                               causal and shard == rank, scale)
+        if world > 1:
+            # the accumulators belong to key shard `shard`: pass them on; after
+            # `world` rotations each is back with its owner
+            yield ("start", list(acc), list(acc_n))
+            yield ("wait",)
+            acc, acc_n = acc_n, acc
+            if s < world - 1:
+                kv = kv_n
+    dq = ops.bwd_finish(ws, q, scale)
+    return dq, ops.to_bf16(acc[0]), ops.to_bf16(acc[1])
+
+
+# ---------------------------------------------------------------- runners
+
+
+def _peer(group, group_rank):
+    import torch.distributed as dist
+    return group_rank if group is None else dist.get_global_rank(group, group_rank)
+
+
+def run_nccl(program, group=None):
+    """Drive one rank's program with torch.distributed point-to-point
+    operations (NCCL for CUDA tensors): "start" posts isend to rank+1 and irecv
+    from rank-1 for each tensor; "wait" makes the current stream wait for
+    all posted operations."""
+    import torch.distributed as dist
+    rank = dist.get_rank(group)
+    world = dist.get_world_size(group)
+    nxt, prv = _peer(group, (rank + 1) % world), _peer(group, (rank - 1) % world)
+    pending = []
+    try:
+        req = next(program)
+        while True:
+            if req[0] == "start":
+                ops = []
+                for snd, rcv in zip(req[1], req[2]):
+                    ops.append(dist.P2POp(dist.isend, snd, nxt, group))
+                    ops.append(dist.P2POp(dist.irecv, rcv, prv, group))
+                pending += dist.batch_isend_irecv(ops)
+            else:
+                for w in pending:
+                    w.wait()
+                pending = []
+            req = program.send(None)
+    except StopIteration as stop:
+        return stop.value
+
+
+def run_local(programs):
+    """Drive the programs of `len(programs)` virtual ranks in lockstep in one
+    process: at each "wait", every rank's posted receive buffers are filled,
+    by device copies, from the previous rank's posted send buffers."""
+    G = len(programs)
+    results = [None] * G
+    reqs = []
+    for p in programs:
+        try:
+            reqs.append(next(p))
+        except StopIteration as stop:
+            reqs.append(("done", stop.value))
+    pending = [[] for _ in range(G)]
+    while True:
+        kinds = {r[0] for r in reqs}
+        if kinds == {"done"}:
+            return [r[1] for r in reqs]
+        if len(kinds) != 1:
+            raise RuntimeError(f"ring programs out of step: {sorted(kinds)}")
+        kind = kinds.pop()
+        if kind == "start":
+            for r in range(G):
+                pending[r].append((reqs[r][1], reqs[r][2]))
+        else:
+            for r in range(G):
+                src = pending[(r - 1) % G]
+                for (snd, _), (_, rcv) in zip(src, pending[r]):
+                    for a, b in zip(snd, rcv):
+                        b.copy_(a)
+            pending = [[] for _ in range(G)]
+        nxt = []
+        for r, p in enumerate(programs):
+            try:
+                nxt.append(p.send(None))
+            except StopIteration as stop:
+                nxt.append(("done", stop.value))
+        reqs = nxt
+
+
+def local_ring_attention(q, k, v, dO, causal: bool, scale: float, world: int, ops=None):
+    """Forward and backward of attention over the whole [B, H, N, d] inputs,
+    computed as a ring of `world` virtual ranks on this device (N divisible by
+    world).  Returns (O, LSE, dQ, dK, dV) for the whole sequence."""
+    N = q.shape[2]
+    if N % world:
+        raise ValueError("sequence length must be divisible by the ring size")
+    n = N // world
+    sl = [slice(r * n, (r + 1) * n) for r in range(world)]
+    shard = lambda t, r: t[:, :, sl[r]].contiguous()  # noqa: E731
+    fwd = run_local([forward_program(shard(q, r), shard(k, r), shard(v, r), causal, scale, r,
+                                     world, ops) for r in range(world)])
+    bwd = run_local([backward_program(shard(q, r), shard(k, r), shard(v, r), fwd[r][0],
+                                      fwd[r][1], shard(dO, r), causal, scale, r, world, ops)
+                     for r in range(world)])
+    cat = lambda xs: torch.cat(xs, dim=2)  # noqa: E731
+    return (cat([f[0] for f in fwd]), cat([f[1] for f in fwd]), cat([b[0] for b in bwd]),
+            cat([b[1] for b in bwd]), cat([b[2] for b in bwd]))

@@ -134,6 +134,56 @@ fa_status fa_bwd_dq_convert(void* dq, int B, int H, int N, int d, float scale,
                             void* stream);
 
 /*
+ * Sequence sharding across devices (Ring Attention with Blockwise
+ * Transformers, abstract: each device keeps its query block while key/value
+ * blocks travel around a ring of devices, overlapped with the blockwise
+ * attention).  Each (query shard, key/value shard) pair is an ordinary
+ * fa_fwd / fa_bwd problem of the shard length; the calls below fold the
+ * pairs' results together.
+ *
+ * fa_lse_merge -- fold one partial attention result into a running one.
+ *   o_acc    [rows, d] fp32, read unless init, written: the running O.
+ *   lse_acc  [rows] fp32 (natural log), likewise: the running LSE.
+ *   o_part   [rows, d] bf16 and lse_part [rows] fp32: attention of the same
+ *            query rows over a key set disjoint from the ones already folded
+ *            in (as fa_fwd writes them).
+ *   o_out    [rows, d] bf16 or NULL: receives bf16(merged O) as well.
+ *   init     1: the accumulator takes the partial as it is; 0: merge,
+ *            O = (w_a O_acc + w_b O_part) / (w_a + w_b), w = exp(LSE - max),
+ *            LSE = max + log(w_a + w_b) (the online-softmax rescaling of
+ *            iplexlaw blog "Tiling preserves the attention calculation").
+ *   rows = number of query rows (e.g. B*H*N), d in {64, 128}.
+ * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_MISALIGNED,
+ * FA_ERR_CUDA.
+ */
+fa_status fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part,
+                       const float* lse_part, void* o_out, long long rows,
+                       int d, int init, void* stream);
+
+/*
+ * fa_bwd_main_accumulate -- fa_bwd_main that ADDS its dK (times scale) and
+ * dV to fp32 accumulators instead of writing bf16: dk_acc, dv_acc
+ * [B,H,N,d] fp32, 16-byte aligned, read-modify-written by bulk reductions.
+ * With a workspace prepared by fa_bwd_preprocess from the FINAL O and LSE
+ * of the query rows (over all key shards), calling it once per key/value
+ * shard accumulates dQ (in the workspace) and each shard's dK, dV exactly as
+ * the gradient over the union of the shards; fa_bwd_dq_convert then yields
+ * dQ.  Other arguments and errors as fa_bwd_main.
+ */
+fa_status fa_bwd_main_accumulate(const void* q, const void* k, const void* v,
+                                 const void* dO, float* dk_acc, float* dv_acc,
+                                 int B, int H, int N, int d, int causal,
+                                 float scale, void* workspace,
+                                 size_t workspace_bytes, void* stream);
+
+/*
+ * fa_convert_f32_bf16 -- dst[i] = bf16(src[i]) (round to nearest even) for
+ * n elements, n a positive multiple of 8; both 16-byte aligned.
+ */
+fa_status fa_convert_f32_bf16(const float* src, void* dst, long long n,
+                              void* stream);
+
+/*
  * fa_bwd_noalloc -- fa_bwd for callers that cannot allocate device memory.
  * (No counterpart in the paper; it is a packaging choice of this library.)
  *   Some callers have no way to hand fa_bwd a workspace: a plugin inside a host

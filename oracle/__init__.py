@@ -196,3 +196,48 @@ def ref_fwd_decode(q, k, v, causal: bool, scale: float, lib=None):
     if rc:
         raise MemoryError("oracle: allocation failed")
     return o, lse
+
+
+# ---------------------------------------------------------------- ring steps
+#
+# Ring Attention with Blockwise Transformers (abstract): the sequence is
+# spread over devices, each keeps its query block while key/value blocks
+# travel, and every block's attention is folded into the running result.
+# The two functions below are the per-step arithmetic of that scheme written
+# out in plain numpy (fp64); they are used to check the ring's host logic.
+
+def ref_lse_merge(o_a, lse_a, o_b, lse_b):
+    """Attention over the union of two disjoint key sets from the results over
+    each: with M = max(lse_a, lse_b) and w = exp(lse - M),
+    O = (w_a O_a + w_b O_b) / (w_a + w_b) and LSE = M + log(w_a + w_b)
+    (the rescaling of the online softmax, iplexlaw blog "Tiling preserves the
+    attention calculation").  o_*: [..., d], lse_*: [...] (natural log)."""
+    o_a, lse_a, o_b, lse_b = (np.asarray(x, dtype=np.float64) for x in (o_a, lse_a, o_b, lse_b))
+    m = np.maximum(lse_a, lse_b)
+    wa = np.exp(lse_a - m)
+    wb = np.exp(lse_b - m)
+    o = (wa[..., None] * o_a + wb[..., None] * o_b) / (wa + wb)[..., None]
+    return o, m + np.log(wa + wb)
+
+
+def ref_grads_given_stats(q, k, v, dO, lse, D, causal: bool, scale: float):
+    """dQ, dK, dV of one (query block, key block) pair when the softmax
+    normaliser and D come from the whole row: P = exp(scale q.k - lse) over
+    this block's keys, dP = dO V^T, dS = P * (dP - D), dQ = scale dS K,
+    dK = scale dS^T Q, dV = P^T dO.  causal: key j of the block visible to
+    query i iff j <= i (the block on the diagonal).  Summed over the key
+    blocks of a row these are the gradient over all its keys.
+    q, dO: [B,H,Nq,d]; k, v: [B,H,Nk,d]; lse, D: [B,H,Nq]."""
+    q, k, v, dO, lse, D = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dO, lse, D))
+    s = scale * np.einsum("bhid,bhjd->bhij", q, k)
+    if causal:
+        nq, nk = s.shape[-2], s.shape[-1]
+        hidden = np.arange(nk)[None, :] > np.arange(nq)[:, None]
+        s = np.where(hidden, -np.inf, s)
+    p = np.exp(s - lse[..., None])
+    dp = np.einsum("bhid,bhjd->bhij", dO, v)
+    ds = p * (dp - D[..., None])
+    dq = scale * np.einsum("bhij,bhjd->bhid", ds, k)
+    dk = scale * np.einsum("bhij,bhid->bhjd", ds, q)
+    dv = np.einsum("bhij,bhid->bhjd", p, dO)
+    return dq, dk, dv

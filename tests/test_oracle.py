@@ -522,3 +522,81 @@ def test_decode_closed_forms():
         np.testing.assert_allclose(la, lb, atol=0)
     with pytest.raises(ValueError):
         oracle.ref_fwd_decode(q, k[:, :, :5], v[:, :, :5], True, 0.7)
+
+
+# ----------------------------------------------------------------------------
+# ring steps: the log-sum-exp merge and gradients under whole-row statistics
+# ----------------------------------------------------------------------------
+
+def test_lse_merge_against_brute_force():
+    """Merging brute-force attention over two disjoint key sets reproduces
+    brute-force attention over their union (no max shift, 50 digits)."""
+    q, k, v, _ = rng_inputs(600, 1, 1, 3, 4)
+    _, k2, v2, _ = rng_inputs(601, 1, 1, 7, 4)
+    kk = np.concatenate([k[0, 0], k2[0, 0]])
+    vv = np.concatenate([v[0, 0], v2[0, 0]])
+    for a in (1, 3, 6):
+        oa, la = brute_decode(q[0, 0], kk[:a], vv[:a], False, 0.9)
+        ob, lb = brute_decode(q[0, 0], kk[a:], vv[a:], False, 0.9)
+        o_all, l_all = brute_decode(q[0, 0], kk, vv, False, 0.9)
+        o, l = oracle.ref_lse_merge(oa, la, ob, lb)
+        assert rel_err(o, o_all) <= 1e-13 and rel_err(l, l_all) <= 1e-13
+        # either order, and a three-way split folded left to right
+        o2, l2 = oracle.ref_lse_merge(ob, lb, oa, la)
+        assert rel_err(o2, o_all) <= 1e-13 and rel_err(l2, l_all) <= 1e-13
+    oa, la = brute_decode(q[0, 0], kk[:2], vv[:2], False, 0.9)
+    ob, lb = brute_decode(q[0, 0], kk[2:5], vv[2:5], False, 0.9)
+    oc, lc = brute_decode(q[0, 0], kk[5:], vv[5:], False, 0.9)
+    o, l = oracle.ref_lse_merge(*oracle.ref_lse_merge(oa, la, ob, lb), oc, lc)
+    o_all, l_all = brute_decode(q[0, 0], kk, vv, False, 0.9)
+    assert rel_err(o, o_all) <= 1e-13 and rel_err(l, l_all) <= 1e-13
+
+
+def test_lse_merge_reproduces_sharded_causal_attention():
+    """The ring decomposition of causal attention: query shard r attends to key
+    shards j < r in full and to shard r causally; merging the pieces gives
+    ref_fwd over the whole sequence."""
+    q, k, v, _ = rng_inputs(602, 2, 2, 24, 8)
+    o_ref, l_ref = oracle.ref_fwd(q, k, v, True, 0.4)
+    G, n = 3, 8
+    for r in range(G):
+        qs = q[:, :, r * n:(r + 1) * n]
+        acc = None
+        for j in range(r + 1):
+            ks, vs = k[:, :, j * n:(j + 1) * n], v[:, :, j * n:(j + 1) * n]
+            part = oracle.ref_fwd(qs, ks, vs, j == r, 0.4)
+            acc = part if acc is None else oracle.ref_lse_merge(*acc, *part)
+        assert rel_err(acc[0], o_ref[:, :, r * n:(r + 1) * n]) <= 1e-12
+        assert rel_err(acc[1], l_ref[:, :, r * n:(r + 1) * n]) <= 1e-12
+
+
+def test_grads_given_stats_sum_to_full_gradient():
+    """Per-shard gradients under the whole rows' LSE and D add up to ref_bwd
+    (itself pinned to numerical derivatives above); with one block they are
+    ref_bwd."""
+    q, k, v, dO = rng_inputs(603, 1, 2, 24, 8)
+    for causal in (False, True):
+        o, lse = oracle.ref_fwd(q, k, v, causal, 0.35)
+        D = np.sum(o * dO, axis=-1)
+        rq, rk, rv, _ = oracle.ref_bwd(q, k, v, dO, causal, 0.35)
+        gq, gk, gv = oracle.ref_grads_given_stats(q, k, v, dO, lse, D, causal, 0.35)
+        assert rel_err(gq, rq) <= 1e-12 and rel_err(gk, rk) <= 1e-12 and rel_err(gv, rv) <= 1e-12
+        G, n = 3, 8
+        dq = np.zeros_like(q)
+        dk = np.zeros_like(k)
+        dv = np.zeros_like(v)
+        for r in range(G):
+            rs = slice(r * n, (r + 1) * n)
+            for j in range(G):
+                if causal and j > r:
+                    continue
+                js = slice(j * n, (j + 1) * n)
+                a, b, c = oracle.ref_grads_given_stats(
+                    q[:, :, rs], k[:, :, js], v[:, :, js], dO[:, :, rs], lse[:, :, rs],
+                    D[:, :, rs], causal and j == r, 0.35)
+                dq[:, :, rs] += a
+                dk[:, :, js] += b
+                dv[:, :, js] += c
+        assert rel_err(dq, rq) <= 1e-12, causal
+        assert rel_err(dk, rk) <= 1e-12, causal
+        assert rel_err(dv, rv) <= 1e-12, causal
