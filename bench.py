@@ -52,6 +52,14 @@ WORKLOADS = {
                                            dist="normal", seed=3),
 }
 
+# Forward with e4m3 Q, K (fa_fwd_qk8): the 16k-token sweep point at d=128.
+QK8_WORKLOADS = {
+    "fwd_qk8_sweep_N8192_d128_causal": dict(B=2, H=16, N=8192, d=128, causal=True,
+                                            dist="normal", seed=2),
+    "fwd_qk8_sweep_N8192_d128_noncausal": dict(B=2, H=16, N=8192, d=128, causal=False,
+                                               dist="normal", seed=2),
+}
+
 # Sequence-sharded (ring) attention, G virtual ranks on one GPU: the long
 # single-sequence shape split into G shards of N/G tokens.
 RING_WORKLOADS = {
@@ -857,6 +865,114 @@ def ring_arm(args, w, wname):
     return 0
 
 
+# ---------------------------------------------------------------- e4m3 scores
+
+
+def qk8_arm(args, w, wname):
+    """Forward only: fa_fwd_qk8 (e4m3 Q, K; bf16 V) timed beside fa_fwd on the
+    dequantised bf16 inputs.  S = QK^T runs at the e4m3 rate and P V at the
+    bf16 rate, so the roofline peak is the harmonic mix of the two: half the
+    FLOPs at 2x the measured bf16 peak (the nominal e4m3:bf16 ratio of 2),
+    half at 1x, i.e. 4/3 of the bf16 peak."""
+    import torch
+
+    import exact_attention_109_b200 as fa
+    from exact_attention_109_b200.inputs import attention_inputs, default_scale, to_e4m3
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        print(json.dumps({"metric": METRIC, "error": "e4m3 workloads run on one GPU"}))
+        return 1
+    torch.cuda.set_device(0)
+    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+    scale = default_scale(d)
+    host = attention_inputs(B, H, N, d, w["seed"], w["dist"])
+    q8, qs = to_e4m3(host["q"])
+    k8, ks = to_e4m3(host["k"])
+    q8d, k8d, v = q8.cuda(), k8.cuda(), host["v"].cuda()
+    qd = (q8.to(torch.float32) * qs).to(torch.bfloat16).cuda()
+    kd = (k8.to(torch.float32) * ks).to(torch.bfloat16).cuda()
+    o = torch.empty_like(v)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    s = torch.cuda.current_stream()
+
+    def step():
+        st = fa.fa_fwd_qk8(q8d.data_ptr(), k8d.data_ptr(), v.data_ptr(), qs, ks, o.data_ptr(),
+                           lse.data_ptr(), B, H, N, d, int(causal), scale, s.cuda_stream)
+        if st != fa.FA_OK:
+            raise fa.FaError(st, "qk8 step")
+
+    def bf16_step():
+        fa.attention_forward(qd, kd, v, causal, scale, out=o, lse=lse)
+
+    for _ in range(args.warmup):
+        step()
+        bf16_step()
+    torch.cuda.synchronize()
+    K = args.steps
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    with ClockSampler(0) as clk:
+        time.sleep(0.3)
+        torch.cuda.synchronize()
+        e[0].record(s)
+        for _ in range(K):
+            step()
+        e[1].record(s)
+        for _ in range(K):
+            bf16_step()
+        e[2].record(s)
+        torch.cuda.synchronize()
+    if fa.fa_get_device_error() != fa.FA_OK:
+        raise RuntimeError("qk8 timed region: device error")
+    ms = e[0].elapsed_time(e[1]) / K
+    bf16_ms = e[1].elapsed_time(e[2]) / K
+    flops = fwd_flops(w)
+    value = flops / (ms * 1e-3) / 1e12
+    # end to end: q8, k8, v in from pinned host memory, O and LSE out
+    pin = [q8.pin_memory(), k8.pin_memory(), host["v"].pin_memory()]
+    dst = [torch.empty_like(q8d), torch.empty_like(k8d), torch.empty_like(v)]
+    oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    Ke = max(4, min(K, 20))
+    e[0].record(s)
+    for _ in range(Ke):
+        for a, b in zip(pin, dst):
+            b.copy_(a, non_blocking=True)
+        fa.attention_forward_qk8(dst[0], dst[1], dst[2], qs, ks, causal, scale, out=o, lse=lse)
+        oh.copy_(o, non_blocking=True)
+        lh.copy_(lse, non_blocking=True)
+    e[3].record(s)
+    torch.cuda.synchronize()
+    e2e = flops / (e[0].elapsed_time(e[3]) / Ke * 1e-3) / 1e12
+    peaks = load_peaks()
+    mixed_peak = peaks["bf16_tflops"] * 4.0 / 3.0
+    cpu = None
+    if not args.no_cpu_baseline:
+        val, tcpu, heads, cores = oracle_whole_heads(w, 20.0)
+        cpu = {"value": val / 3.5, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"oracle ref_fwd + ref_bwd on {heads} whole heads, {tcpu:.1f} s, "
+                         f"credited the forward's share of the FLOPs"}
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "e4m3 QK^T, bf16 PV", "data": "synthetic",
+        "config": dict(workload_config(w, wname), **{"pass": "fwd", "quant": "per-tensor e4m3 "
+                       "Q, K (descale = amax / 448)",
+                       "l2": f"no flush: per-step working set {(2 + 4) * B * H * N * d / 1e6:.0f} MB"}),
+        "bf16_fwd_tflops": flops / (bf16_ms * 1e-3) / 1e12,
+        "speedup_vs_bf16": bf16_ms / ms,
+        "roofline": {"kernel": "fa_fwd_kernel<128, causal, e4m3>", "bound": "tensor",
+                     "achieved": value, "peak": mixed_peak, "unit": "TFLOP/s",
+                     "frac": value / mixed_peak,
+                     "peak_source": f"{peaks['source']} bf16 burst x 4/3 (half the FLOPs at the "
+                                    f"nominal 2x e4m3 rate)", "traffic": None},
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin),
+                "d2h_bytes_per_step": oh.numel() * 2 + lh.numel() * 4},
+        "gpu_launches": K, "clocks": clk.summary()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -864,11 +980,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS)
-                    + sorted(RING_WORKLOADS),
+                    + sorted(RING_WORKLOADS) + sorted(QK8_WORKLOADS),
                     default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.workload in QK8_WORKLOADS:
+        if args.impl == "reference":
+            return reference_arm(args, QK8_WORKLOADS[args.workload], args.workload)
+        return qk8_arm(args, QK8_WORKLOADS[args.workload], args.workload)
     if args.workload in RING_WORKLOADS:
         if args.impl == "reference":
             return reference_arm(args, RING_WORKLOADS[args.workload], args.workload)

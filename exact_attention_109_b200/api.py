@@ -78,6 +78,8 @@ def library():
     lib.fa_bwd_main_accumulate.restype = i
     lib.fa_convert_f32_bf16.argtypes = [vp, vp, ll, vp]
     lib.fa_convert_f32_bf16.restype = i
+    lib.fa_fwd_qk8.argtypes = [vp, vp, vp, f, f, vp, vp, i, i, i, i, i, f, vp]
+    lib.fa_fwd_qk8.restype = i
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
     lib.fa_selftest_wait_timeout.restype = i
     lib.fa_get_device_error.argtypes = [vp]
@@ -175,6 +177,13 @@ def fa_decode_split_plan(B: int, H: int, Nq: int, Nk: int, d: int, sm_count: int
                                         ctypes.byref(qg), ctypes.byref(ns),
                                         ctypes.byref(ch))
     return st, qg.value, ns.value, ch.value
+
+
+def fa_fwd_qk8(q: int, k: int, v: int, q_descale: float, k_descale: float, o: int, lse: int,
+               B: int, H: int, N: int, d: int, causal: int, scale: float, stream: int = 0) -> int:
+    """Raw C call: forward pass with e4m3 Q and K; returns the status."""
+    return library().fa_fwd_qk8(q, k, v, float(q_descale), float(k_descale), o, lse, B, H, N,
+                                d, int(causal), float(scale), stream or None)
 
 
 def fa_lse_merge(o_acc: int, lse_acc: int, o_part: int, lse_part: int, o_out: int,
@@ -295,4 +304,23 @@ def attention_decode(q, k, v, causal: bool, scale: float, n_keys: int | None = N
     _check(fa_fwd_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, Nq, Nk,
                          kv_rows, d, int(causal), scale, ws_ptr, ws_bytes, s),
            "fa_fwd_decode")
+    return out, lse
+
+
+def attention_forward_qk8(q8, k8, v, q_descale: float, k_descale: float, causal: bool,
+                          scale: float, out=None, lse=None, stream=None):
+    """O, LSE = fa_fwd_qk8: q8, k8 CUDA float8_e4m3fn [B,H,N,d] with their
+    per-tensor dequantisation factors, v CUDA bf16 [B,H,N,d]."""
+    B, H, N, d = _shape(q8)
+    _require({"q8": q8, "k8": k8}, (B, H, N, d), torch.float8_e4m3fn, q8.device)
+    _require({"v": v}, (B, H, N, d), torch.bfloat16, q8.device)
+    if out is None:
+        out = torch.empty(v.shape, dtype=torch.bfloat16, device=v.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=v.device)
+    _require({"out": out}, (B, H, N, d), torch.bfloat16, q8.device)
+    _require({"lse": lse}, (B, H, N), torch.float32, q8.device)
+    s = (stream or torch.cuda.current_stream(v.device)).cuda_stream
+    _check(fa_fwd_qk8(_ptr(q8), _ptr(k8), _ptr(v), q_descale, k_descale, _ptr(out), _ptr(lse),
+                      B, H, N, d, int(causal), scale, s), "fa_fwd_qk8")
     return out, lse

@@ -133,6 +133,14 @@ fa_status device_setup(int* dev_out, unsigned int** err_out) {
                              fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
         ok &= prepare_kernel(fa::fa_bwd_main_kernel<128, true>, fa::BwdTraits<128>::SMEM_BYTES,
                              fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd_kernel<128, false, true>,
+                             fa::FwdTraits<128, true>::SMEM_BYTES,
+                             fa::FwdTraits<128, true>::NUM_THREADS,
+                             fa::FwdTraits<128, true>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd_kernel<128, true, true>,
+                             fa::FwdTraits<128, true>::SMEM_BYTES,
+                             fa::FwdTraits<128, true>::NUM_THREADS,
+                             fa::FwdTraits<128, true>::REG_BUDGET);
         ok &= cudaDeviceGetAttribute(&s.sm_count, cudaDevAttrMultiProcessorCount, dev) ==
               cudaSuccess;
         ok &= prepare_decode<64>(s.dec_occ[0]);
@@ -183,14 +191,14 @@ bool encode_bf16(CUtensorMap* map, const void* base, int d, int N, long long bh,
     return encode_3d(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, box_rows);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool QK8 = false>
 cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& mo, const fa::FwdParams& prm, long long bh,
                        cudaStream_t stream) {
-    using T = fa::FwdTraits<D>;
+    using T = fa::FwdTraits<D, QK8>;
     const long long grid = bh * prm.n_qpairs;
-    fa::fa_fwd_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), T::NUM_THREADS, T::SMEM_BYTES,
-                                   stream>>>(mq, mk, mv, mo, prm);
+    fa::fa_fwd_kernel<D, CAUSAL, QK8><<<static_cast<unsigned>(grid), T::NUM_THREADS,
+                                        T::SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
     return cudaGetLastError();
 }
 
@@ -243,6 +251,44 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     else
         e = causal ? launch_fwd<128, true>(mq, mk, mv, mo, prm, bh, s)
                    : launch_fwd<128, false>(mq, mk, mv, mo, prm, bh, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_qk8(const void* q, const void* k, const void* v, float q_descale,
+                     float k_descale, void* o, float* lse, int B, int H, int N, int d,
+                     int causal, float scale, void* stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    fa_status st = check_sizes(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (!(std::isfinite(q_descale) && q_descale > 0.f && std::isfinite(k_descale) &&
+          k_descale > 0.f))
+        return FA_ERR_INVALID_ARG;
+    const float sl2 = scale * q_descale * k_descale * 1.4426950408889634f;
+    if (!(std::isfinite(sl2) && sl2 > 0.f)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_MISALIGNED;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    int dev;
+    unsigned int* err;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    if (!load_encode()) return FA_ERR_CUDA;
+    const long long bh = static_cast<long long>(B) * H;
+    CUtensorMap mq, mk, mv, mo;
+    if (!encode_3d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
+        !encode_3d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
+        !encode_bf16(&mv, v, d, N, bh, 128) || !encode_bf16(&mo, o, d, N, bh, 32))
+        return FA_ERR_CUDA;
+    fa::FwdParams prm;
+    prm.lse = lse;
+    prm.err = err;
+    prm.N = N;
+    prm.n_qpairs = (N + 255) / 256;
+    prm.bh_count = static_cast<int>(bh);
+    prm.scale_log2 = sl2;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = causal ? launch_fwd<128, true, true>(mq, mk, mv, mo, prm, bh, s)
+                                 : launch_fwd<128, false, true>(mq, mk, mv, mo, prm, bh, s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

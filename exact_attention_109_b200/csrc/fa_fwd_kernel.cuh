@@ -32,19 +32,30 @@
 
 namespace fa {
 
-template <int D>
+// QK8: Q and K are e4m3 (one byte per element) and S = Q K^T runs as a
+// kind::f8f6f4 MMA at twice the bf16 rate; P and V stay bf16.
+template <int D, bool QK8 = false>
 struct FwdTraits {
     static_assert(D == 64 || D == 128, "head dim");
+    static_assert(!QK8 || D == 128, "e4m3 scores need 128-byte rows (d = 128)");
     static constexpr int BM = 128;                  // query rows per tile
     static constexpr int BN = 128;                  // key rows per block
     static constexpr int TILES = 2;                 // query tiles per CTA
-    static constexpr int CHUNKS = D / 64;           // 128-byte swizzle column chunks
+    static constexpr int CHUNKS = D / 64;           // 128-byte swizzle column chunks (bf16)
     static constexpr int CHUNK_BYTES = 128 * 128;   // 128 rows x 128 B
     static constexpr int TILE_BYTES = BM * D * 2;   // one 128-row bf16 tile
+    static constexpr int QK_ELEM = QK8 ? 1 : 2;     // bytes per Q / K element
+    static constexpr int QK_CHUNKS = D * QK_ELEM / 128;
+    static constexpr int QK_CHUNK_COLS = 128 / QK_ELEM;  // elements per swizzle chunk row
+    static constexpr int QK_TILE_BYTES = BM * D * QK_ELEM;
+    static constexpr int S_KSTEPS = D * QK_ELEM / 32;    // 32-byte K steps of S = Q K^T
     static constexpr int NSLOT = (D == 128) ? 4 : 8;
     static constexpr int Q_OFF = 0;
-    static constexpr int KV_OFF = Q_OFF + TILES * TILE_BYTES;
-    static constexpr int BAR_OFF = KV_OFF + NSLOT * TILE_BYTES;
+    static constexpr int KV_OFF = Q_OFF + TILES * QK_TILE_BYTES;
+    // O staging for the epilogue: in the tile's own Q buffer when that holds
+    // a bf16 tile, else in a region of its own (an e4m3 Q tile is half size).
+    static constexpr int OST_OFF = KV_OFF + NSLOT * TILE_BYTES;
+    static constexpr int BAR_OFF = OST_OFF + (QK8 ? TILES * TILE_BYTES : 0);
     // q, full[NSLOT], empty[NSLOT], s_full[2], p_ready[2], o_final[2], mma_done
     static constexpr int NBAR = 1 + 2 * NSLOT + 2 + 2 + 2 + 1;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
@@ -57,7 +68,7 @@ struct FwdTraits {
     static constexpr uint32_t REG_CONTROL = 72;
     static constexpr int REG_BUDGET = 128 * (2 * REG_SOFTMAX + REG_CONTROL);
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, 0, 0);
+    static constexpr uint32_t IDESC_S = QK8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, 0, 0);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
     static constexpr float TAU = 8.0f;  // deferred-rescale threshold (log2 units)
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -108,12 +119,12 @@ __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], f
     lr += b0 + b1;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool QK8 = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const FwdParams p) {
-    using T = FwdTraits<D>;
+    using T = FwdTraits<D, QK8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -184,11 +195,11 @@ __global__ void __launch_bounds__(384, 1)
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             bool ok = true;
-            mbar_arrive_expect_tx(bar_q, T::TILES * T::TILE_BYTES);
+            mbar_arrive_expect_tx(bar_q, T::TILES * T::QK_TILE_BYTES);
             for (int t = 0; t < T::TILES; ++t)
-                for (int c = 0; c < T::CHUNKS; ++c)
-                    tma_load_3d(smem + T::Q_OFF + t * T::TILE_BYTES + c * T::CHUNK_BYTES, &tmQ,
-                                bar_q, c * 64, q0 + 128 * t, bh);
+                for (int c = 0; c < T::QK_CHUNKS; ++c)
+                    tma_load_3d(smem + T::Q_OFF + t * T::QK_TILE_BYTES + c * T::CHUNK_BYTES,
+                                &tmQ, bar_q, c * T::QK_CHUNK_COLS, q0 + 128 * t, bh);
             int issued = 0;
             for (int j = 0; j < n1 && ok; ++j) {
                 for (int h = 0; h < 2; ++h) {  // 0: K_j, 1: V_j
@@ -199,11 +210,13 @@ __global__ void __launch_bounds__(384, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[slot], T::TILE_BYTES);
+                    mbar_arrive_expect_tx(&full[slot], h ? T::TILE_BYTES : T::QK_TILE_BYTES);
                     uint8_t* dst = smem + T::KV_OFF + slot * T::TILE_BYTES;
-                    for (int c = 0; c < T::CHUNKS; ++c)
-                        tma_load_3d(dst + c * T::CHUNK_BYTES, h ? &tmV : &tmK, &full[slot], c * 64,
-                                    j * T::BN, bh);
+                    const int nch = h ? T::CHUNKS : T::QK_CHUNKS;
+                    const int ccols = h ? 64 : T::QK_CHUNK_COLS;
+                    for (int c = 0; c < nch; ++c)
+                        tma_load_3d(dst + c * T::CHUNK_BYTES, h ? &tmV : &tmK, &full[slot],
+                                    c * ccols, j * T::BN, bh);
                     ++issued;
                 }
             }
@@ -224,14 +237,18 @@ __global__ void __launch_bounds__(384, 1)
                 return kv_base + static_cast<uint32_t>((idx % T::NSLOT) * T::TILE_BYTES);
             };
             auto slot_par = [&](int idx) { return static_cast<uint32_t>((idx / T::NSLOT) & 1); };
-            // S_t = Q_t K^T : M=128, N=128, K=D, both operands K-major.
+            // S_t = Q_t K^T : M=128, N=128, K=D, both operands K-major;
+            // each MMA consumes 32 bytes of every row (16 bf16 or 32 e4m3).
             auto mma_s = [&](int t, uint32_t k_addr) {
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k) {
+                for (int k = 0; k < T::S_KSTEPS; ++k) {
                     const uint32_t off = (k >> 2) * T::CHUNK_BYTES + (k & 3) * 32;
-                    const uint64_t a = sdesc_sw128(q_base + t * T::TILE_BYTES + off, 16, 1024);
+                    const uint64_t a = sdesc_sw128(q_base + t * T::QK_TILE_BYTES + off, 16, 1024);
                     const uint64_t b = sdesc_sw128(k_addr + off, 16, 1024);
-                    umma_ss(tmem + 128u * t, a, b, T::IDESC_S, k > 0 ? 1u : 0u);
+                    if constexpr (QK8)
+                        umma_ss_f8(tmem + 128u * t, a, b, T::IDESC_S, k > 0 ? 1u : 0u);
+                    else
+                        umma_ss(tmem + 128u * t, a, b, T::IDESC_S, k > 0 ? 1u : 0u);
                 }
             };
             // O_t += P_t V : M=128, N=D, K=128; P from TMEM, V MN-major.
@@ -385,8 +402,10 @@ __global__ void __launch_bounds__(384, 1)
             const float inv_l = 1.0f / lr;
             const float lse_val = (m + log2f(l)) * 0.6931471805599453f;
             // Stage O (bf16, 128-byte swizzle) in this tile's Q buffer, which
-            // no MMA reads any more, then store this warp's 32 rows by TMA.
-            uint8_t* stage = smem + T::Q_OFF + t * T::TILE_BYTES + lg * 32 * 128;
+            // no MMA reads any more (e4m3 scores: in the staging region),
+            // then store this warp's 32 rows by TMA.
+            uint8_t* stage = smem + (QK8 ? T::OST_OFF : T::Q_OFF) + t * T::TILE_BYTES +
+                             lg * 32 * 128;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 uint32_t o[32];

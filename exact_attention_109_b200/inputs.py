@@ -71,6 +71,17 @@ def decode_inputs(B: int, H: int, Nq: int, Nk: int, d: int, seed: int,
     return out
 
 
+def to_e4m3(x: torch.Tensor):
+    """Per-tensor e4m3 (float8_e4m3fn) quantisation of a CPU tensor, as a
+    caller of the 8-bit score path would do it: descale = max|x| / 448 (the
+    largest finite e4m3 value), x8 = round-to-nearest(x / descale).  Returns
+    (x8, descale); the dequantised tensor is x8 * descale."""
+    amax = float(x.abs().max())
+    descale = float(np.float32(amax / 448.0)) if amax > 0 else 1.0
+    x8 = (x.to(torch.float32) / descale).to(torch.float8_e4m3fn)
+    return x8, descale
+
+
 def default_scale(d: int) -> float:
     """1/sqrt(d) rounded to fp32, the value both sides receive."""
     return float(np.float32(1.0 / math.sqrt(d)))

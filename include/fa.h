@@ -74,6 +74,28 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o,
                  float scale, void* stream);
 
 /*
+ * fa_fwd_qk8 -- forward pass with 8-bit float scores (low-precision attention
+ * on Blackwell tensor cores, in the manner of SageAttention, whose
+ * Blackwell work the pages cite: the QK^T product is quantised, P V stays in
+ * 16 bits).
+ *   q, k     [B,H,N,d] e4m3 (1 byte per element, OCP FP8 E4M3), read only,
+ *            with per-tensor dequantisation factors q_descale, k_descale
+ *            (finite, > 0): the attention is that of q_descale * q and
+ *            k_descale * k.
+ *   v        [B,H,N,d] bf16.  o, lse as fa_fwd.
+ * S = Q K^T runs as tcgen05.mma kind::f8f6f4 (e4m3 x e4m3, fp32 accumulate,
+ * exact products) at twice the bf16 rate; the descales fold into the softmax
+ * scale; P is rounded to bf16 for P V exactly as in fa_fwd.  For inputs that
+ * are e4m3 values, the result is fa_fwd's on the dequantised Q and K, within
+ * the same tolerances.  Supported: d = 128.  Other conventions and errors as
+ * fa_fwd (FA_ERR_UNSUPPORTED for d != 128).
+ */
+fa_status fa_fwd_qk8(const void* q, const void* k, const void* v,
+                     float q_descale, float k_descale, void* o, float* lse,
+                     int B, int H, int N, int d, int causal, float scale,
+                     void* stream);
+
+/*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs:
  * an fp32 dQ accumulator [B,H,Npad,d] plus two fp32 row vectors [B,H,Npad]
  * (log2-scaled LSE and D = rowsum(dO * O)), Npad = N rounded up to 128.
