@@ -60,6 +60,13 @@ QK8_WORKLOADS = {
                                                dist="normal", seed=2),
 }
 
+# Additive score bias (fa_fwd_bias / fa_bwd_bias): 16k tokens, a bias shared
+# by the batch ([1, H, N, N] bf16), dBias [B, H, N, N] written.
+BIAS_WORKLOADS = {
+    "fwd_bwd_bias_B4_H16_N4096_d128_causal": dict(B=4, H=16, N=4096, d=128, causal=True,
+                                                  dist="normal", seed=2),
+}
+
 # Sequence-sharded (ring) attention, G virtual ranks on one GPU: the long
 # single-sequence shape split into G shards of N/G tokens.
 RING_WORKLOADS = {
@@ -973,6 +980,108 @@ def qk8_arm(args, w, wname):
     return 0
 
 
+# ---------------------------------------------------------------- bias
+
+
+def bias_arm(args, w, wname):
+    """One step = fa_fwd_bias + fa_bwd_bias (with dBias), timed beside the
+    plain fa_fwd + fa_bwd on the same q, k, v, dO.  TFLOP/s by the same
+    convention; the bias adds HBM traffic (the bias read in both passes,
+    dBias written), reported as bias_bytes_per_step."""
+    import torch
+
+    import exact_attention_109_b200 as fa
+    from exact_attention_109_b200.inputs import attention_inputs, default_scale
+
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        print(json.dumps({"metric": METRIC, "error": "bias workloads run on one GPU"}))
+        return 1
+    torch.cuda.set_device(0)
+    B, H, N, d, causal = w["B"], w["H"], w["N"], w["d"], w["causal"]
+    scale = default_scale(d)
+    host = attention_inputs(B, H, N, d, w["seed"], w["dist"], with_dout=True)
+    q, k, v, dO = (host[x].cuda() for x in ("q", "k", "v", "dO"))
+    g = torch.Generator().manual_seed(w["seed"] + 7)
+    bias = (torch.randn((1, H, N, N), generator=g) * 2).to(torch.bfloat16).cuda()
+    ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream()
+
+    ob, lb = fa.attention_forward_bias(q, k, v, bias, causal, scale)
+
+    def fwd_only():
+        fa.attention_forward_bias(q, k, v, bias, causal, scale, out=ob, lse=lb)
+
+    def bwd_only():
+        fa.attention_backward_bias(q, k, v, bias, ob, lb, dO, causal, scale, workspace=ws)
+
+    def step():
+        fwd_only()
+        bwd_only()
+
+    def plain_step():
+        o, lse = fa.attention_forward(q, k, v, causal, scale)
+        fa.attention_backward(q, k, v, o, lse, dO, causal, scale, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+        plain_step()
+    torch.cuda.synchronize()
+    K = args.steps
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    with ClockSampler(0) as clk:
+        time.sleep(0.3)
+        torch.cuda.synchronize()
+        e[0].record(s)
+        for _ in range(K):
+            step()
+        e[1].record(s)
+        for _ in range(K):
+            plain_step()
+        e[2].record(s)
+        torch.cuda.synchronize()
+    f = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    f[0].record(s)
+    for _ in range(K):
+        fwd_only()
+    f[1].record(s)
+    for _ in range(K):
+        bwd_only()
+    f[2].record(s)
+    torch.cuda.synchronize()
+    if fa.fa_get_device_error() != fa.FA_OK:
+        raise RuntimeError("bias timed region: device error")
+    ms, plain_ms = e[0].elapsed_time(e[1]) / K, e[1].elapsed_time(e[2]) / K
+    pass_ms = {"fwd_bias": f[0].elapsed_time(f[1]) / K, "bwd_bias": f[1].elapsed_time(f[2]) / K}
+    flops = 3.5 * fwd_flops(w)
+    value = flops / (ms * 1e-3) / 1e12
+    frac_causal = 0.5 if causal else 1.0
+    bias_bytes = int(B * H * N * N * 2 * frac_causal * 3)  # read twice, dBias written once
+    peaks = load_peaks()
+    cpu = None
+    if not args.no_cpu_baseline:
+        val, tcpu, heads, cores = oracle_whole_heads(w, 20.0)
+        cpu = {"value": val, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": f"oracle ref_fwd + ref_bwd (without the bias term) on {heads} whole "
+                         f"heads, {tcpu:.1f} s"}
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(workload_config(w, wname), **{
+            "pass": "fwd+bwd with additive bias", "bias": f"[1, {H}, {N}, {N}] bf16",
+            "l2": "no flush: per-step working set > 126 MB"}),
+        "plain_fwd_bwd_tflops": flops / (plain_ms * 1e-3) / 1e12,
+        "bias_overhead": ms / plain_ms - 1.0, "bias_bytes_per_step": bias_bytes,
+        "pass_ms": pass_ms,
+        "roofline": {"kernel": "whole step (fa_fwd_kernel, fa_bwd_main_kernel with bias)",
+                     "bound": "tensor", "achieved": value, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": value / peaks["bf16_tflops"],
+                     "peak_source": f"{peaks['source']} (burst)", "traffic": None},
+        "cpu_baseline": cpu, "e2e": None, "gpu_launches": 4 * K,
+        "clocks": clk.summary()}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -980,11 +1089,16 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS) + sorted(DECODE_WORKLOADS)
-                    + sorted(RING_WORKLOADS) + sorted(QK8_WORKLOADS),
+                    + sorted(RING_WORKLOADS) + sorted(QK8_WORKLOADS)
+                    + sorted(BIAS_WORKLOADS),
                     default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.workload in BIAS_WORKLOADS:
+        if args.impl == "reference":
+            return reference_arm(args, BIAS_WORKLOADS[args.workload], args.workload)
+        return bias_arm(args, BIAS_WORKLOADS[args.workload], args.workload)
     if args.workload in QK8_WORKLOADS:
         if args.impl == "reference":
             return reference_arm(args, QK8_WORKLOADS[args.workload], args.workload)

@@ -80,6 +80,11 @@ def library():
     lib.fa_convert_f32_bf16.restype = i
     lib.fa_fwd_qk8.argtypes = [vp, vp, vp, f, f, vp, vp, i, i, i, i, i, f, vp]
     lib.fa_fwd_qk8.restype = i
+    lib.fa_fwd_bias.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp]
+    lib.fa_fwd_bias.restype = i
+    lib.fa_bwd_bias.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
+                                f, vp, sz, vp]
+    lib.fa_bwd_bias.restype = i
     lib.fa_selftest_wait_timeout.argtypes = [ctypes.c_uint, vp]
     lib.fa_selftest_wait_timeout.restype = i
     lib.fa_get_device_error.argtypes = [vp]
@@ -184,6 +189,24 @@ def fa_fwd_qk8(q: int, k: int, v: int, q_descale: float, k_descale: float, o: in
     """Raw C call: forward pass with e4m3 Q and K; returns the status."""
     return library().fa_fwd_qk8(q, k, v, float(q_descale), float(k_descale), o, lse, B, H, N,
                                 d, int(causal), float(scale), stream or None)
+
+
+def fa_fwd_bias(q: int, k: int, v: int, bias: int, o: int, lse: int, B: int, H: int, N: int,
+                d: int, bias_batch: int, bias_heads: int, causal: int, scale: float,
+                stream: int = 0) -> int:
+    """Raw C call: forward pass with an additive score bias."""
+    return library().fa_fwd_bias(q, k, v, bias, o, lse, B, H, N, d, int(bias_batch),
+                                 int(bias_heads), int(causal), float(scale), stream or None)
+
+
+def fa_bwd_bias(q: int, k: int, v: int, bias: int, o: int, lse: int, dO: int, dq: int, dk: int,
+                dv: int, dbias: int, B: int, H: int, N: int, d: int, bias_batch: int,
+                bias_heads: int, causal: int, scale: float, workspace: int,
+                workspace_bytes: int, stream: int = 0) -> int:
+    """Raw C call: backward pass with an additive score bias (dbias may be 0)."""
+    return library().fa_bwd_bias(q, k, v, bias, o, lse, dO, dq, dk, dv, dbias or None, B, H, N,
+                                 d, int(bias_batch), int(bias_heads), int(causal), float(scale),
+                                 workspace, int(workspace_bytes), stream or None)
 
 
 def fa_lse_merge(o_acc: int, lse_acc: int, o_part: int, lse_part: int, o_out: int,
@@ -324,3 +347,51 @@ def attention_forward_qk8(q8, k8, v, q_descale: float, k_descale: float, causal:
     _check(fa_fwd_qk8(_ptr(q8), _ptr(k8), _ptr(v), q_descale, k_descale, _ptr(out), _ptr(lse),
                       B, H, N, d, int(causal), scale, s), "fa_fwd_qk8")
     return out, lse
+
+
+def _bias_flags(bias, B, H, N):
+    if bias.dim() != 4 or tuple(bias.shape[2:]) != (N, N) or bias.shape[0] not in (1, B) \
+            or bias.shape[1] not in (1, H):
+        raise ValueError(f"bias: expected [B or 1, H or 1, {N}, {N}], got {tuple(bias.shape)}")
+    if bias.dtype != torch.bfloat16 or not bias.is_contiguous():
+        raise TypeError("bias: expected a contiguous bf16 tensor")
+    return int(bias.shape[0] == B and B > 1), int(bias.shape[1] == H and H > 1)
+
+
+def attention_forward_bias(q, k, v, bias, causal: bool, scale: float, out=None, lse=None,
+                           stream=None):
+    """O, LSE = fa_fwd_bias: scores scale * q.k + bias for CUDA bf16 [B,H,N,d]
+    q, k, v and a bf16 bias [B or 1, H or 1, N, N]."""
+    B, H, N, d = _shape(q)
+    _require({"q": q, "k": k, "v": v}, (B, H, N, d), torch.bfloat16, q.device)
+    bb, bh_ = _bias_flags(bias, B, H, N)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _require({"out": out}, (B, H, N, d), torch.bfloat16, q.device)
+    _require({"lse": lse}, (B, H, N), torch.float32, q.device)
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    _check(fa_fwd_bias(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(out), _ptr(lse), B, H, N, d,
+                       bb, bh_, int(causal), scale, s), "fa_fwd_bias")
+    return out, lse
+
+
+def attention_backward_bias(q, k, v, bias, out, lse, dO, causal: bool, scale: float,
+                            want_dbias: bool = True, workspace=None, stream=None):
+    """dQ, dK, dV, dBias (or None) = fa_bwd_bias(...); dBias is [B,H,N,N] bf16."""
+    B, H, N, d = _shape(q)
+    _require({"q": q, "k": k, "v": v, "out": out, "dO": dO}, (B, H, N, d), torch.bfloat16,
+             q.device)
+    _require({"lse": lse}, (B, H, N), torch.float32, q.device)
+    bb, bh_ = _bias_flags(bias, B, H, N)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    dbias = torch.empty((B, H, N, N), dtype=torch.bfloat16, device=q.device) if want_dbias \
+        else None
+    need = fa_bwd_workspace_size(B, H, N, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    s = (stream or torch.cuda.current_stream(q.device)).cuda_stream
+    _check(fa_bwd_bias(_ptr(q), _ptr(k), _ptr(v), _ptr(bias), _ptr(out), _ptr(lse), _ptr(dO),
+                       _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dbias) if dbias is not None else 0,
+                       B, H, N, d, bb, bh_, int(causal), scale, _ptr(workspace),
+                       workspace.numel() * workspace.element_size(), s), "fa_bwd_bias")
+    return dq, dk, dv, dbias

@@ -101,6 +101,15 @@ bool prepare_decode(int (&occ)[3]) {
            prepare_decode_one<D, 4>(&occ[2]);
 }
 
+template <int D>
+bool prepare_fwd_bias() {
+    using T = fa::FwdTraits<D, false, true>;
+    return prepare_kernel(fa::fa_fwd_kernel<D, false, false, true>, T::SMEM_BYTES,
+                          T::NUM_THREADS, T::REG_BUDGET) &&
+           prepare_kernel(fa::fa_fwd_kernel<D, true, false, true>, T::SMEM_BYTES, T::NUM_THREADS,
+                          T::REG_BUDGET);
+}
+
 // One-time per-device set-up: architecture check, error-word address, and
 // the shared-memory opt-in of every kernel.  Returns FA_OK or an error.
 fa_status device_setup(int* dev_out, unsigned int** err_out) {
@@ -141,6 +150,19 @@ fa_status device_setup(int* dev_out, unsigned int** err_out) {
                              fa::FwdTraits<128, true>::SMEM_BYTES,
                              fa::FwdTraits<128, true>::NUM_THREADS,
                              fa::FwdTraits<128, true>::REG_BUDGET);
+        ok &= prepare_fwd_bias<64>() && prepare_fwd_bias<128>();
+        ok &= prepare_kernel(fa::fa_bwd_main_kernel<64, false, true>,
+                             fa::BwdTraits<64>::SMEM_BYTES, fa::BwdTraits<64>::NUM_THREADS,
+                             fa::BwdTraits<64>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_bwd_main_kernel<64, true, true>,
+                             fa::BwdTraits<64>::SMEM_BYTES, fa::BwdTraits<64>::NUM_THREADS,
+                             fa::BwdTraits<64>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_bwd_main_kernel<128, false, true>,
+                             fa::BwdTraits<128>::SMEM_BYTES, fa::BwdTraits<128>::NUM_THREADS,
+                             fa::BwdTraits<128>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_bwd_main_kernel<128, true, true>,
+                             fa::BwdTraits<128>::SMEM_BYTES, fa::BwdTraits<128>::NUM_THREADS,
+                             fa::BwdTraits<128>::REG_BUDGET);
         ok &= cudaDeviceGetAttribute(&s.sm_count, cudaDevAttrMultiProcessorCount, dev) ==
               cudaSuccess;
         ok &= prepare_decode<64>(s.dec_occ[0]);
@@ -191,15 +213,30 @@ bool encode_bf16(CUtensorMap* map, const void* base, int d, int N, long long bh,
     return encode_3d(map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, d, N, bh, 64, box_rows);
 }
 
-template <int D, bool CAUSAL, bool QK8 = false>
+// mb: the bias tensor map (BIAS); other variants get any map, unused.
+template <int D, bool CAUSAL, bool QK8 = false, bool BIAS = false>
 cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                       const CUtensorMap& mo, const fa::FwdParams& prm, long long bh,
-                       cudaStream_t stream) {
-    using T = fa::FwdTraits<D, QK8>;
+                       const CUtensorMap& mo, const CUtensorMap& mb, const fa::FwdParams& prm,
+                       long long bh, cudaStream_t stream) {
+    using T = fa::FwdTraits<D, QK8, BIAS>;
     const long long grid = bh * prm.n_qpairs;
-    fa::fa_fwd_kernel<D, CAUSAL, QK8><<<static_cast<unsigned>(grid), T::NUM_THREADS,
-                                        T::SMEM_BYTES, stream>>>(mq, mk, mv, mo, prm);
+    fa::fa_fwd_kernel<D, CAUSAL, QK8, BIAS><<<static_cast<unsigned>(grid), T::NUM_THREADS,
+                                              T::SMEM_BYTES, stream>>>(mq, mk, mv, mo, mb, prm);
     return cudaGetLastError();
+}
+
+fa::FwdParams fwd_params(float* lse, unsigned int* err, int N, long long bh, int H, float sl2) {
+    fa::FwdParams prm;
+    prm.lse = lse;
+    prm.err = err;
+    prm.N = N;
+    prm.n_qpairs = (N + 255) / 256;
+    prm.bh_count = static_cast<int>(bh);
+    prm.scale_log2 = sl2;
+    prm.H = H;
+    prm.bias_batch = 0;
+    prm.bias_heads = 0;
+    return prm;
 }
 
 }  // namespace
@@ -236,21 +273,15 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     if (!encode_bf16(&mq, q, d, N, bh, 128) || !encode_bf16(&mk, k, d, N, bh, 128) ||
         !encode_bf16(&mv, v, d, N, bh, 128) || !encode_bf16(&mo, o, d, N, bh, 32))
         return FA_ERR_CUDA;
-    fa::FwdParams prm;
-    prm.lse = lse;
-    prm.err = err;
-    prm.N = N;
-    prm.n_qpairs = (N + 255) / 256;
-    prm.bh_count = static_cast<int>(bh);
-    prm.scale_log2 = scale * 1.4426950408889634f;
+    const fa::FwdParams prm = fwd_params(lse, err, N, bh, H, scale * 1.4426950408889634f);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (d == 64)
-        e = causal ? launch_fwd<64, true>(mq, mk, mv, mo, prm, bh, s)
-                   : launch_fwd<64, false>(mq, mk, mv, mo, prm, bh, s);
+        e = causal ? launch_fwd<64, true>(mq, mk, mv, mo, mo, prm, bh, s)
+                   : launch_fwd<64, false>(mq, mk, mv, mo, mo, prm, bh, s);
     else
-        e = causal ? launch_fwd<128, true>(mq, mk, mv, mo, prm, bh, s)
-                   : launch_fwd<128, false>(mq, mk, mv, mo, prm, bh, s);
+        e = causal ? launch_fwd<128, true>(mq, mk, mv, mo, mo, prm, bh, s)
+                   : launch_fwd<128, false>(mq, mk, mv, mo, mo, prm, bh, s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -279,16 +310,48 @@ fa_status fa_fwd_qk8(const void* q, const void* k, const void* v, float q_descal
         !encode_3d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
         !encode_bf16(&mv, v, d, N, bh, 128) || !encode_bf16(&mo, o, d, N, bh, 32))
         return FA_ERR_CUDA;
-    fa::FwdParams prm;
-    prm.lse = lse;
-    prm.err = err;
-    prm.N = N;
-    prm.n_qpairs = (N + 255) / 256;
-    prm.bh_count = static_cast<int>(bh);
-    prm.scale_log2 = sl2;
+    const fa::FwdParams prm = fwd_params(lse, err, N, bh, H, sl2);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const cudaError_t e = causal ? launch_fwd<128, true, true>(mq, mk, mv, mo, prm, bh, s)
-                                 : launch_fwd<128, false, true>(mq, mk, mv, mo, prm, bh, s);
+    const cudaError_t e = causal ? launch_fwd<128, true, true>(mq, mk, mv, mo, mo, prm, bh, s)
+                                 : launch_fwd<128, false, true>(mq, mk, mv, mo, mo, prm, bh, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_bias(const void* q, const void* k, const void* v, const void* bias, void* o,
+                      float* lse, int B, int H, int N, int d, int bias_batch, int bias_heads,
+                      int causal, float scale, void* stream) {
+    if (!q || !k || !v || !bias || !o || !lse) return FA_ERR_INVALID_ARG;
+    fa_status st = check_sizes(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if ((bias_batch != 0 && bias_batch != 1) || (bias_heads != 0 && bias_heads != 1) ||
+        (causal != 0 && causal != 1))
+        return FA_ERR_INVALID_ARG;
+    if (N % 8 != 0) return FA_ERR_UNSUPPORTED;  // bias rows must be 16-byte multiples
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(bias) || !aligned16(o) ||
+        !aligned16(lse))
+        return FA_ERR_MISALIGNED;
+    int dev;
+    unsigned int* err;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    if (!load_encode()) return FA_ERR_CUDA;
+    const long long bh = static_cast<long long>(B) * H;
+    const long long nb = static_cast<long long>(bias_batch ? B : 1) * (bias_heads ? H : 1);
+    CUtensorMap mq, mk, mv, mo, mb;
+    if (!encode_bf16(&mq, q, d, N, bh, 128) || !encode_bf16(&mk, k, d, N, bh, 128) ||
+        !encode_bf16(&mv, v, d, N, bh, 128) || !encode_bf16(&mo, o, d, N, bh, 32) ||
+        !encode_3d(&mb, bias, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, N, nb, 64, 128))
+        return FA_ERR_CUDA;
+    fa::FwdParams prm = fwd_params(lse, err, N, bh, H, scale * 1.4426950408889634f);
+    prm.bias_batch = bias_batch;
+    prm.bias_heads = bias_heads;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (d == 64)
+        e = causal ? launch_fwd<64, true, false, true>(mq, mk, mv, mo, mb, prm, bh, s)
+                   : launch_fwd<64, false, false, true>(mq, mk, mv, mo, mb, prm, bh, s);
+    else
+        e = causal ? launch_fwd<128, true, false, true>(mq, mk, mv, mo, mb, prm, bh, s)
+                   : launch_fwd<128, false, false, true>(mq, mk, mv, mo, mb, prm, bh, s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -334,7 +397,9 @@ fa_status bwd_pre_impl(const void* o, const float* lse, const void* dO, int B, i
 
 fa_status bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, void* dk,
                         void* dv, int B, int H, int N, int d, int causal, float scale,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+                        void* workspace, size_t workspace_bytes, void* stream,
+                        const void* bias = nullptr, void* dbias = nullptr, int bias_batch = 0,
+                        int bias_heads = 0) {
     if (!q || !k || !v || !dO || !dk || !dv) return FA_ERR_INVALID_ARG;
     if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
     fa::BwdWorkspace ws;
@@ -358,16 +423,21 @@ fa_status bwd_main_impl(const void* q, const void* k, const void* v, const void*
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int ibh = static_cast<int>(bh);
     cudaError_t e;
-    if (d == 64)
-        e = causal ? fa::launch_bwd_main<64, true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
-                                                   macc, err, s)
-                   : fa::launch_bwd_main<64, false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
-                                                    macc, err, s);
-    else
-        e = causal ? fa::launch_bwd_main<128, true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
-                                                    macc, err, s)
-                   : fa::launch_bwd_main<128, false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk,
-                                                     mdv, macc, err, s);
+#define FA_BWD_MAIN(DD, CC, BB)                                                            \
+    fa::launch_bwd_main<DD, CC, BB>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv, macc, err, s, \
+                                    0, bias, dbias, H, bias_batch, bias_heads)
+    if (bias) {
+        if (d == 64)
+            e = causal ? FA_BWD_MAIN(64, true, true) : FA_BWD_MAIN(64, false, true);
+        else
+            e = causal ? FA_BWD_MAIN(128, true, true) : FA_BWD_MAIN(128, false, true);
+    } else {
+        if (d == 64)
+            e = causal ? FA_BWD_MAIN(64, true, false) : FA_BWD_MAIN(64, false, false);
+        else
+            e = causal ? FA_BWD_MAIN(128, true, false) : FA_BWD_MAIN(128, false, false);
+    }
+#undef FA_BWD_MAIN
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -520,6 +590,47 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
         return st;
     if ((st = bwd_main_impl(q, k, v, dO, dk, dv, B, H, N, d, causal, scale, workspace,
                             workspace_bytes, stream)) != FA_OK)
+        return st;
+    return bwd_convert_impl(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_bwd_bias(const void* q, const void* k, const void* v, const void* bias,
+                      const void* o, const float* lse, const void* dO, void* dq, void* dk,
+                      void* dv, void* dbias, int B, int H, int N, int d, int bias_batch,
+                      int bias_heads, int causal, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+    if (!q || !k || !v || !bias || !o || !lse || !dO || !dq || !dk || !dv || !workspace)
+        return FA_ERR_INVALID_ARG;
+    fa_status st = check_sizes(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if ((bias_batch != 0 && bias_batch != 1) || (bias_heads != 0 && bias_heads != 1) ||
+        (causal != 0 && causal != 1))
+        return FA_ERR_INVALID_ARG;
+    if (N % 8 != 0) return FA_ERR_UNSUPPORTED;
+    if (workspace_bytes < fa::bwd_workspace_bytes(static_cast<long long>(B) * H, N, d))
+        return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(bias) || !aligned16(o) ||
+        !aligned16(lse) || !aligned16(dO) || !aligned16(dq) || !aligned16(dk) || !aligned16(dv) ||
+        (dbias && !aligned16(dbias)) || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return FA_ERR_MISALIGNED;
+    int dev;
+    unsigned int* err;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    if (!load_encode()) return FA_ERR_CUDA;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    // With the causal mask the main kernel never visits the key blocks past
+    // a query row's own block, whose gradient is zero: write those zeros.
+    if (dbias && causal) {
+        const long long rows = static_cast<long long>(B) * H * N;
+        fa::fa_dbias_zero_upper_kernel<<<static_cast<unsigned>((rows + 7) / 8), 256, 0, s>>>(
+            static_cast<__nv_bfloat16*>(dbias), N, rows);
+        if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+    }
+    if ((st = bwd_pre_impl(o, lse, dO, B, H, N, d, workspace, workspace_bytes, stream)) != FA_OK)
+        return st;
+    if ((st = bwd_main_impl(q, k, v, dO, dk, dv, B, H, N, d, causal, scale, workspace,
+                            workspace_bytes, stream, bias, dbias, bias_batch, bias_heads)) !=
+        FA_OK)
         return st;
     return bwd_convert_impl(dq, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }

@@ -117,6 +117,24 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(
     *reinterpret_cast<uint4*>(dq + e) = out;
 }
 
+// ------------------------------------------------------------------ dBias
+//
+// Causal dBias: the main kernel writes every (query, key) pair of the key
+// blocks it visits, from the query block holding the block's first key
+// onwards (hidden pairs inside as 0).  The pairs it never visits are those
+// of query row q with keys from the next 128-key block on: this kernel
+// zeroes exactly those, [128 (floor(q / 128) + 1), N) of every row, with
+// 16-byte stores (N % 8 == 0).  One warp per row.
+__global__ void __launch_bounds__(256) fa_dbias_zero_upper_kernel(__nv_bfloat16* dbias, int N,
+                                                                   long long rows) {
+    const long long row = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
+    if (row >= rows) return;
+    const int q = static_cast<int>(row % N);
+    const int c0 = (q / kBwdBN + 1) * kBwdBN;
+    uint4* dst = reinterpret_cast<uint4*>(dbias + row * N);
+    for (int c = c0 / 8 + (threadIdx.x & 31); c < N / 8; c += 32) dst[c] = make_uint4(0, 0, 0, 0);
+}
+
 // ------------------------------------------------------------------ 2. main
 
 template <int D>
@@ -181,11 +199,20 @@ struct BwdParams {
     int n_kv;        // ceil(N / 128)
     int n_q;         // ceil(N / 64)
     int accum;       // 0: write bf16 dK, dV; 1: add them to fp32 accumulators
+    // Additive score bias (null: none): bias [Bb][Hb][N][N] bf16, with
+    // Bb = B when bias_batch (else 1) and Hb = H when bias_heads (else 1);
+    // dbias (null: not wanted) [B][H][N][N] bf16 receives dS.
+    const __nv_bfloat16* bias;
+    __nv_bfloat16* dbias;
+    int H;
+    int bias_batch;
+    int bias_heads;
     float scale;
     float scale_log2;
 };
 
-template <int D, bool CAUSAL>
+// BIAS: an additive score bias (and optionally its gradient), see BwdParams.
+template <int D, bool CAUSAL, bool BIAS = false>
 __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
     const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -401,9 +428,49 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
         const int kv_row = j * T::BN + r;
         const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
         const float sl2 = p.scale_log2;
+        // Bias and its gradient are read and written straight from / to HBM:
+        // for a fixed query row the 32 lanes of a warp touch 32 consecutive
+        // keys (64 contiguous bytes) per instruction.
+        const __nv_bfloat16* bias_base = nullptr;
+        if (BIAS) {
+            const int bb = bh / p.H, hh = bh % p.H;
+            const long long bz = static_cast<long long>(p.bias_batch ? bb : 0) *
+                                     (p.bias_heads ? p.H : 1) + (p.bias_heads ? hh : 0);
+            bias_base = p.bias + bz * N * N;
+        }
+        __nv_bfloat16* dbias_base =
+            BIAS && p.dbias ? p.dbias + static_cast<long long>(bh) * N * N : nullptr;
+        // Bias b[q][key] of a block's 32 query columns.  The loads run one
+        // block ahead: block k+1's are issued at the top of block k (raw
+        // 16-bit values, one register each) and packed at its end, so an HBM
+        // round trip never stalls a block.
+        unsigned short braw[32];
+        uint32_t bpk[16];
+        auto bias_load = [&](int kk) {
+            const int q0 = (qb0 + kk) * T::BM + 32 * g;
+            const unsigned short* bp = reinterpret_cast<const unsigned short*>(bias_base) +
+                                       static_cast<long long>(q0) * N + kv_row;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                braw[e] = (kv_row < N && q0 + e < N) ? __ldg(bp + static_cast<long long>(e) * N)
+                                                     : static_cast<unsigned short>(0);
+        };
+        auto bias_pack = [&]() {
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                bpk[e] = static_cast<uint32_t>(braw[2 * e]) |
+                         (static_cast<uint32_t>(braw[2 * e + 1]) << 16);
+        };
+        if constexpr (BIAS) {
+            bias_load(0);
+            bias_pack();
+        }
         bool ok = true;
         for (int k = 0; k < n; ++k) {
             const int b = k & 1;
+            if constexpr (BIAS) {
+                if (k + 1 < n) bias_load(k + 1);
+            }
             ok = __all_sync(0xffffffffu, mbar_wait(&sdp_full[b], (k >> 1) & 1, st));
             if (!ok) break;
             tc_fence_after();
@@ -431,7 +498,13 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
 #pragma unroll
                 for (int h = 0; h < 4; ++h) {
                     const int e = 4 * e4 + h;
-                    float x = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, -lsv[h]));
+                    float arg = -lsv[h];
+                    if constexpr (BIAS) {
+                        const uint32_t w = bpk[e >> 1];
+                        const float bv = __uint_as_float((e & 1) ? (w & 0xffff0000u) : (w << 16));
+                        arg = fmaf(bv, 1.4426950408889634f, arg);
+                    }
+                    float x = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, arg));
                     if (CAUSAL && e < masked) x = 0.f;
                     pr[h] = x;
                     ds[h] = x * (__uint_as_float(dp[e]) - dsv_[h]);
@@ -440,6 +513,16 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
                 pk[2 * e4 + 1] = pack_bf16x2(pr[2], pr[3]);
                 dk[2 * e4] = pack_bf16x2(ds[0], ds[1]);
                 dk[2 * e4 + 1] = pack_bf16x2(ds[2], ds[3]);
+            }
+            if (BIAS && dbias_base && kv_row < N) {
+                // dBias = dS, rounded to bf16 as for the dQ and dK MMAs
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (qrow0 + e < N)
+                        *reinterpret_cast<unsigned short*>(
+                            dbias_base + static_cast<long long>(qrow0 + e) * N + kv_row) =
+                            static_cast<unsigned short>((e & 1) ? (dk[e >> 1] >> 16)
+                                                                : (dk[e >> 1] & 0xffffu));
             }
             // P^T then dS^T over this warpgroup's own S columns (A operands of
             // the dV and dK MMAs).
@@ -455,6 +538,9 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&pds_ready[b]);
+            if constexpr (BIAS) {
+                if (k + 1 < n) bias_pack();
+            }
         }
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(kv_done, 0, st));
         if (ok && p.accum) {
@@ -593,12 +679,14 @@ cudaError_t launch_bwd_pre(const void* o, const float* lse, const void* dO, int 
 }
 
 // Stage 2: dK, dV and the fp32 dQ accumulation (needs stage 1's workspace).
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool BIAS = false>
 cudaError_t launch_bwd_main(int bh, int N, float scale, const BwdWorkspace& ws,
                             const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                             const CUtensorMap& mdo, const CUtensorMap& mdk,
                             const CUtensorMap& mdv, const CUtensorMap& macc, unsigned int* err,
-                            cudaStream_t s, int accum = 0) {
+                            cudaStream_t s, int accum = 0, const void* bias = nullptr,
+                            void* dbias = nullptr, int H = 1, int bias_batch = 0,
+                            int bias_heads = 0) {
     using T = BwdTraits<D>;
     BwdParams prm;
     prm.lse2 = ws.lse2;
@@ -610,10 +698,16 @@ cudaError_t launch_bwd_main(int bh, int N, float scale, const BwdWorkspace& ws,
     prm.n_kv = (N + T::BN - 1) / T::BN;
     prm.n_q = (N + T::BM - 1) / T::BM;
     prm.accum = accum;
+    prm.bias = static_cast<const __nv_bfloat16*>(bias);
+    prm.dbias = static_cast<__nv_bfloat16*>(dbias);
+    prm.H = H;
+    prm.bias_batch = bias_batch;
+    prm.bias_heads = bias_heads;
     prm.scale = scale;
     prm.scale_log2 = scale * 1.4426950408889634f;
     const long long grid = static_cast<long long>(bh) * prm.n_kv;
-    fa_bwd_main_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), T::NUM_THREADS, T::SMEM_BYTES, s>>>(
+    fa_bwd_main_kernel<D, CAUSAL, BIAS><<<static_cast<unsigned>(grid), T::NUM_THREADS,
+                                          T::SMEM_BYTES, s>>>(
         mq, mk, mv, mdo, mdk, mdv, macc, prm);
     return cudaGetLastError();
 }

@@ -34,10 +34,13 @@ namespace fa {
 
 // QK8: Q and K are e4m3 (one byte per element) and S = Q K^T runs as a
 // kind::f8f6f4 MMA at twice the bf16 rate; P and V stay bf16.
-template <int D, bool QK8 = false>
+// BIAS: an additive bf16 score bias b_ij, one [128 x 128] tile per query
+// tile and key block, brought in by TMA.
+template <int D, bool QK8 = false, bool BIAS = false>
 struct FwdTraits {
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(!QK8 || D == 128, "e4m3 scores need 128-byte rows (d = 128)");
+    static_assert(!(QK8 && BIAS), "one variant at a time");
     static constexpr int BM = 128;                  // query rows per tile
     static constexpr int BN = 128;                  // key rows per block
     static constexpr int TILES = 2;                 // query tiles per CTA
@@ -49,20 +52,27 @@ struct FwdTraits {
     static constexpr int QK_CHUNK_COLS = 128 / QK_ELEM;  // elements per swizzle chunk row
     static constexpr int QK_TILE_BYTES = BM * D * QK_ELEM;
     static constexpr int S_KSTEPS = D * QK_ELEM / 32;    // 32-byte K steps of S = Q K^T
-    static constexpr int NSLOT = (D == 128) ? 4 : 8;
+    static constexpr int NSLOT = (D == 128) ? (BIAS ? 3 : 4) : 8;
     static constexpr int Q_OFF = 0;
     static constexpr int KV_OFF = Q_OFF + TILES * QK_TILE_BYTES;
     // O staging for the epilogue: in the tile's own Q buffer when that holds
     // a bf16 tile, else in a region of its own (an e4m3 Q tile is half size).
     static constexpr int OST_OFF = KV_OFF + NSLOT * TILE_BYTES;
-    static constexpr int BAR_OFF = OST_OFF + (QK8 ? TILES * TILE_BYTES : 0);
-    // q, full[NSLOT], empty[NSLOT], s_full[2], p_ready[2], o_final[2], mma_done
-    static constexpr int NBAR = 1 + 2 * NSLOT + 2 + 2 + 2 + 1;
+    // Bias tiles (BIAS): one [128 rows][128 keys] bf16 tile per query tile,
+    // two 64-key swizzle chunks each, single-buffered: the softmax reads its
+    // row of the tile right after the scores, long before the next one.
+    static constexpr int BIAS_TILE = BM * BN * 2;
+    static constexpr int BIAS_OFF = OST_OFF + (QK8 ? TILES * TILE_BYTES : 0);
+    static constexpr int BAR_OFF = BIAS_OFF + (BIAS ? TILES * BIAS_TILE : 0);
+    // q, full[NSLOT], empty[NSLOT], s_full[2], p_ready[2], o_final[2],
+    // mma_done, bias_full[2], bias_empty[2]
+    static constexpr int NBAR = 1 + 2 * NSLOT + 2 + 2 + 2 + 1 + 4;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
     static constexpr int NUM_THREADS = 384;  // 3 warpgroups; warps 10-11 idle
     static constexpr int MMA_WARP = 8;
     static constexpr int LOAD_WARP = 9;
+    static constexpr int BIAS_WARP = 10;
     // Register split: softmax warpgroups grow, the MMA/TMA warpgroup shrinks.
     static constexpr uint32_t REG_SOFTMAX = 216;
     static constexpr uint32_t REG_CONTROL = 72;
@@ -81,6 +91,9 @@ struct FwdParams {
     int n_qpairs;          // ceil(N / 256)
     int bh_count;          // B * H
     float scale_log2;      // scale * log2(e)
+    int H;                 // heads (to split b*H + h)
+    int bias_batch;        // bias varies with the batch index (else shared)
+    int bias_heads;        // bias varies with the head index (else shared)
 };
 
 // One softmax row over a 128-key block: p = exp2(s * scale*log2(e) - m) in
@@ -119,12 +132,12 @@ __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], f
     lr += b0 + b1;
 }
 
-template <int D, bool CAUSAL, bool QK8 = false>
+template <int D, bool CAUSAL, bool QK8 = false, bool BIAS = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                  const FwdParams p) {
-    using T = FwdTraits<D, QK8>;
+                  const __grid_constant__ CUtensorMap tmB, const FwdParams p) {
+    using T = FwdTraits<D, QK8, BIAS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -136,6 +149,8 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* p_ready = s_full + 2;
     uint64_t* o_final = p_ready + 2;
     uint64_t* mma_done = o_final + 2;
+    uint64_t* bias_full = mma_done + 1;
+    uint64_t* bias_empty = bias_full + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::MISC_OFF + 4);
 
@@ -169,6 +184,8 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&s_full[t], 1);
             mbar_init(&p_ready[t], 128);
             mbar_init(&o_final[t], 1);
+            mbar_init(&bias_full[t], 1);
+            mbar_init(&bias_empty[t], 128);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -183,6 +200,7 @@ __global__ void __launch_bounds__(384, 1)
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
         tma_prefetch_desc(&tmO);
+        if (BIAS) tma_prefetch_desc(&tmB);
     }
     tc_fence_before();
     __syncthreads();
@@ -226,6 +244,34 @@ __global__ void __launch_bounds__(384, 1)
                     mbar_wait_bounded(&full[idx % T::NSLOT], (idx / T::NSLOT) & 1);
                 mbar_wait_bounded(bar_q, 0);
             }
+        }
+        __syncwarp();
+      } else if (BIAS && warp == T::BIAS_WARP) {
+        // ------------------------------------------------ bias tile producer
+        if (lane == 0) {
+            const int b = bh / p.H, h = bh % p.H;
+            const int bz = (p.bias_batch ? b : 0) * (p.bias_heads ? p.H : 1) +
+                           (p.bias_heads ? h : 0);
+            int issued[2] = {0, 0};
+            bool ok = true;
+            for (int j = 0; j < n1 && ok; ++j) {
+                for (int t = 0; t < 2; ++t) {
+                    if (j >= (t ? n1 : n0)) continue;
+                    if (j > 0 && !mbar_wait(&bias_empty[t], (j - 1) & 1, st)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&bias_full[t], T::BIAS_TILE);
+                    uint8_t* dst = smem + T::BIAS_OFF + t * T::BIAS_TILE;
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_3d(dst + c * T::CHUNK_BYTES, &tmB, &bias_full[t],
+                                    j * T::BN + 64 * c, q0 + 128 * t, bz);
+                    ++issued[t];
+                }
+            }
+            if (!ok)  // let the copies in flight land before the CTA exits
+                for (int t = 0; t < 2; ++t)
+                    if (issued[t]) mbar_wait_bounded(&bias_full[t], (issued[t] - 1) & 1);
         }
         __syncwarp();
       } else if (warp == T::MMA_WARP) {
@@ -345,6 +391,36 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
             for (int c = 0; c < 4; ++c) tmem_ld32(s_tm + 32u * c, sr[c]);
             tmem_ld_wait();
+            if constexpr (BIAS) {
+                // Scores become t = s * scale*log2(e) + b * log2(e), the
+                // exponent in base 2 (so the rest runs with unit scale).
+                ok = __all_sync(0xffffffffu, mbar_wait(&bias_full[t], j & 1, st));
+                if (!ok) break;
+                const uint8_t* brow = smem + T::BIAS_OFF + t * T::BIAS_TILE + r * 128;
+                const uint64_t sl2x2 = f2_pack(sl2, sl2);
+                const uint64_t lg2x2 = f2_pack(1.4426950408889634f, 1.4426950408889634f);
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {  // keys 8u .. 8u+7
+                    const uint4 bv = *reinterpret_cast<const uint4*>(
+                        brow + (u >> 3) * T::CHUNK_BYTES + (((u & 7) ^ (r & 7)) << 4));
+                    const uint32_t w[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int c = 8 * u + 2 * i;
+                        const uint64_t b2 = f2_pack(__uint_as_float(w[i] << 16),
+                                                    __uint_as_float(w[i] & 0xffff0000u));
+                        const uint64_t s2 = f2_pack(__uint_as_float(sr[c >> 5][c & 31]),
+                                                    __uint_as_float(sr[c >> 5][(c & 31) + 1]));
+                        float t0, t1;
+                        f2_unpack(ffma2(s2, sl2x2, ffma2(b2, lg2x2, 0ull)), t0, t1);
+                        sr[c >> 5][c & 31] = __float_as_uint(t0);
+                        sr[c >> 5][(c & 31) + 1] = __float_as_uint(t1);
+                    }
+                }
+                mbar_arrive(&bias_empty[t]);
+            }
+            constexpr float kUnit = 1.0f;
+            const float sl2e = BIAS ? kUnit : sl2;  // scale still to apply to sr
 
             const int kv0 = j * T::BN;
             // Only the ragged last block and (causal) the diagonal block hold
@@ -369,7 +445,7 @@ __global__ void __launch_bounds__(384, 1)
                     mx[i] = fmaxf(mx[i], __uint_as_float(sr[(c + i) >> 5][(c + i) & 31]));
             mx[0] = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-            const float m_blk = mx[0] * sl2;
+            const float m_blk = mx[0] * sl2e;
             const float m_new = (m_blk > m + T::TAU) ? m_blk : m;
             if (j > 0) {
                 const bool grow = m_new != m;
@@ -390,7 +466,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             m = m_new;
-            softmax_block_exp(sr, sl2, m, s_tm, l, lr);
+            softmax_block_exp(sr, sl2e, m, s_tm, l, lr);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_ready[t]);

@@ -96,6 +96,45 @@ fa_status fa_fwd_qk8(const void* q, const void* k, const void* v,
                      void* stream);
 
 /*
+ * Attention with an additive score bias: S_ij = scale * q_i.k_j + b_ij
+ * (a prior added to the query-key scores, the "attention with bias" of
+ * vision, language and protein-folding models that the pages cite), before
+ * the causal mask and the softmax.
+ *
+ * fa_fwd_bias -- fa_fwd with a bias.
+ *   bias     [Bb, Hb, N, N] bf16, read only: Bb = B if bias_batch else 1,
+ *            Hb = H if bias_heads else 1 (a bias shared by the batch and/or
+ *            the heads, e.g. a relative-position bias).  Row i, column j is
+ *            the bias of query i and key j.  Each row needs at least one
+ *            finite biased score among its visible keys (a bias of -inf
+ *            masks a key).
+ *   lse      includes the bias: LSE_i = ln sum_j exp(scale q_i.k_j + b_ij).
+ *   Needs N % 8 == 0 (each bias row a multiple of 16 bytes), else
+ *   FA_ERR_UNSUPPORTED.  Other arguments, conventions and errors as fa_fwd.
+ */
+fa_status fa_fwd_bias(const void* q, const void* k, const void* v,
+                      const void* bias, void* o, float* lse, int B, int H,
+                      int N, int d, int bias_batch, int bias_heads, int causal,
+                      float scale, void* stream);
+
+/*
+ * fa_bwd_bias -- fa_bwd for fa_fwd_bias (same bias, flags, causal, scale),
+ *   recomputing P = exp(scale q.k + b - LSE).
+ *   dbias    [B, H, N, N] bf16, or NULL: receives the gradient of the bias,
+ *            dS_ij = P_ij (dP_ij - D_i), for every batch and head (sum it over
+ *            the batch / heads yourself when the bias is shared).  With the
+ *            causal mask the hidden entries are written as 0.
+ *   The other arguments, the workspace, conventions and errors are those of
+ *   fa_bwd; N % 8 == 0 as for fa_fwd_bias.
+ */
+fa_status fa_bwd_bias(const void* q, const void* k, const void* v,
+                      const void* bias, const void* o, const float* lse,
+                      const void* dO, void* dq, void* dk, void* dv, void* dbias,
+                      int B, int H, int N, int d, int bias_batch, int bias_heads,
+                      int causal, float scale, void* workspace,
+                      size_t workspace_bytes, void* stream);
+
+/*
  * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs:
  * an fp32 dQ accumulator [B,H,Npad,d] plus two fp32 row vectors [B,H,Npad]
  * (log2-scaled LSE and D = rowsum(dO * O)), Npad = N rounded up to 128.

@@ -241,3 +241,53 @@ def ref_grads_given_stats(q, k, v, dO, lse, D, causal: bool, scale: float):
     dk = scale * np.einsum("bhij,bhid->bhjd", ds, q)
     dv = np.einsum("bhij,bhid->bhjd", p, dO)
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------- score bias
+#
+# Attention with an additive bias matrix on the query-key scores (the
+# "attention with bias" blurb of the pages): s_ij = scale q_i.k_j + b_ij, then
+# the mask, the softmax and P V as before.  Plain numpy, fp64, materialised
+# scores and a two-pass softmax.
+
+def _biased_scores(q, k, bias, causal, scale):
+    q, k, bias = (np.asarray(x, dtype=np.float64) for x in (q, k, bias))
+    s = scale * np.einsum("bhid,bhjd->bhij", q, k) + bias
+    if causal:
+        n = s.shape[-1]
+        s = np.where(np.arange(n)[None, :] > np.arange(n)[:, None], -np.inf, s)
+    return s
+
+
+def ref_fwd_bias(q, k, v, bias, causal: bool, scale: float):
+    """O and LSE (natural log) of softmax(scale Q K^T + bias [+ causal]) V.
+    bias: [Bb, Hb, N, N] with Bb in {1, B}, Hb in {1, H} (broadcast)."""
+    s = _biased_scores(q, k, bias, causal, scale)
+    m = np.max(s, axis=-1, keepdims=True)
+    p = np.exp(s - m)
+    den = np.sum(p, axis=-1, keepdims=True)
+    o = np.einsum("bhij,bhjd->bhid", p / den, np.asarray(v, dtype=np.float64))
+    return o, (m + np.log(den))[..., 0]
+
+
+def ref_bwd_bias(q, k, v, bias, dO, causal: bool, scale: float, o_given=None):
+    """dQ, dK, dV and dBias ([B,H,N,N], per batch and head) of
+    L = sum(O * dO): P = softmax(s), dP = dO V^T, D = rowsum(dO * O),
+    dS = P * (dP - D), dQ = scale dS K, dK = scale dS^T Q, dV = P^T dO,
+    dBias = dS.  o_given: take D from this O (the forward output a backward
+    pass receives) instead of the exact one."""
+    q, k, v, dO = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dO))
+    s = _biased_scores(q, k, bias, causal, scale)
+    m = np.max(s, axis=-1, keepdims=True)
+    p = np.exp(s - m)
+    p = p / np.sum(p, axis=-1, keepdims=True)
+    o = np.einsum("bhij,bhjd->bhid", p, v)
+    if o_given is not None:
+        o = np.asarray(o_given, dtype=np.float64)
+    dp = np.einsum("bhid,bhjd->bhij", dO, v)
+    D = np.sum(dO * o, axis=-1, keepdims=True)
+    ds = p * (dp - D)
+    dq = scale * np.einsum("bhij,bhjd->bhid", ds, k)
+    dk = scale * np.einsum("bhij,bhid->bhjd", ds, q)
+    dv = np.einsum("bhij,bhid->bhjd", p, dO)
+    return dq, dk, dv, ds

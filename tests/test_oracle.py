@@ -600,3 +600,92 @@ def test_grads_given_stats_sum_to_full_gradient():
         assert rel_err(dq, rq) <= 1e-12, causal
         assert rel_err(dk, rk) <= 1e-12, causal
         assert rel_err(dv, rv) <= 1e-12, causal
+
+
+# ----------------------------------------------------------------------------
+# additive score bias
+# ----------------------------------------------------------------------------
+
+def test_bias_zero_and_mask_reduce_to_plain_attention():
+    q, k, v, dO = rng_inputs(700, 2, 3, 9, 4)
+    zero = np.zeros((1, 1, 9, 9))
+    for causal in (False, True):
+        o, l = oracle.ref_fwd_bias(q, k, v, zero, causal, 0.6)
+        o2, l2 = oracle.ref_fwd(q, k, v, causal, 0.6)
+        assert rel_err(o, o2) <= 1e-13 and rel_err(l, l2) <= 1e-13
+        g = oracle.ref_bwd_bias(q, k, v, zero, dO, causal, 0.6)
+        g2 = oracle.ref_bwd(q, k, v, dO, causal, 0.6)
+        for a, b in zip(g[:3], g2[:3]):
+            assert rel_err(a, b) <= 1e-12
+    # a bias of -inf above the diagonal is the causal mask
+    mask = np.where(np.arange(9)[None, :] > np.arange(9)[:, None], -np.inf, 0.0)[None, None]
+    o, l = oracle.ref_fwd_bias(q, k, v, mask, False, 0.6)
+    o2, l2 = oracle.ref_fwd(q, k, v, True, 0.6)
+    assert rel_err(o, o2) <= 1e-13 and rel_err(l, l2) <= 1e-13
+
+
+def test_bias_row_constant_shifts_lse_only():
+    q, k, v, _ = rng_inputs(701, 1, 2, 7, 3)
+    c = np.random.default_rng(1).standard_normal((1, 2, 7, 1)) * 3
+    bias = np.broadcast_to(c, (1, 2, 7, 7)).copy()
+    o, l = oracle.ref_fwd_bias(q, k, v, bias, True, 0.5)
+    o2, l2 = oracle.ref_fwd(q, k, v, True, 0.5)
+    assert rel_err(o, o2) <= 1e-13
+    np.testing.assert_allclose(l, l2 + c[..., 0], atol=1e-13)
+
+
+def test_bias_against_brute_force():
+    q, k, v, _ = rng_inputs(702, 1, 1, 5, 3)
+    bias = np.random.default_rng(2).standard_normal((1, 1, 5, 5)) * 2
+    for causal in (False, True):
+        o, l = oracle.ref_fwd_bias(q, k, v, bias, causal, 0.7)
+        with mp.workdps(50):
+            for i in range(5):
+                keys = range(i + 1) if causal else range(5)
+                w = [mp.exp(mp.mpf(0.7) * mp.fsum(mp.mpf(float(q[0, 0, i, t])) *
+                                                   mp.mpf(float(k[0, 0, j, t])) for t in range(3))
+                            + mp.mpf(float(bias[0, 0, i, j]))) for j in keys]
+                Z = mp.fsum(w)
+                assert abs(float(mp.log(Z)) - l[0, 0, i]) <= 1e-13
+                for t in range(3):
+                    ref = float(mp.fsum(w[a] * mp.mpf(float(v[0, 0, j, t]))
+                                        for a, j in enumerate(keys)) / Z)
+                    assert abs(ref - o[0, 0, i, t]) <= 1e-13
+
+
+def test_bias_against_torch_autograd():
+    """torch's fp64 SDPA with a float additive mask, and autograd for the
+    gradients of q, k, v and the mask (broadcast over the batch)."""
+    q, k, v, dO = rng_inputs(703, 2, 3, 11, 5)
+    bias = np.random.default_rng(3).standard_normal((1, 3, 11, 11))
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    tb = torch.tensor(bias, requires_grad=True)
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=tb, scale=0.45)
+    (out * torch.tensor(dO)).sum().backward()
+    o, _ = oracle.ref_fwd_bias(q, k, v, bias, False, 0.45)
+    dq, dk, dv, db = oracle.ref_bwd_bias(q, k, v, bias, dO, False, 0.45)
+    assert rel_err(o, out.detach().numpy()) <= 1e-12
+    assert rel_err(dq, tq.grad.numpy()) <= 1e-11
+    assert rel_err(dk, tk.grad.numpy()) <= 1e-11
+    assert rel_err(dv, tv.grad.numpy()) <= 1e-11
+    # the broadcast bias's gradient is dBias summed over the batch
+    assert rel_err(db.sum(axis=0, keepdims=True), tb.grad.numpy()) <= 1e-11
+
+
+def test_bias_gradient_by_finite_differences():
+    q, k, v, dO = rng_inputs(704, 1, 1, 6, 3)
+    bias = np.random.default_rng(4).standard_normal((1, 1, 6, 6))
+    _, _, _, db = oracle.ref_bwd_bias(q, k, v, bias, dO, True, 0.8)
+    h = 1e-6
+    for (i, j) in [(0, 0), (3, 1), (5, 5), (5, 2), (2, 2)]:
+        bp, bm = bias.copy(), bias.copy()
+        bp[0, 0, i, j] += h
+        bm[0, 0, i, j] -= h
+        lp = np.sum(oracle.ref_fwd_bias(q, k, v, bp, True, 0.8)[0] * dO)
+        lm = np.sum(oracle.ref_fwd_bias(q, k, v, bm, True, 0.8)[0] * dO)
+        assert abs((lp - lm) / (2 * h) - db[0, 0, i, j]) <= 1e-7
+    assert np.all(db[0, 0][np.triu_indices(6, 1)] == 0)  # hidden pairs
+    # with the exact O passed as o_given nothing changes
+    o, _ = oracle.ref_fwd_bias(q, k, v, bias, True, 0.8)
+    db2 = oracle.ref_bwd_bias(q, k, v, bias, dO, True, 0.8, o_given=o)[3]
+    assert rel_err(db2, db) <= 1e-14
