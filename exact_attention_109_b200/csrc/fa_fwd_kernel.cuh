@@ -100,6 +100,9 @@ struct FwdParams {
 // pairs (f32x2 FFMA for the argument), packed to bf16 and written over the
 // first 64 TMEM columns of S; returns the fp32 sum of p (for the LSE) and of
 // the bf16-rounded p (for normalising O) through two f32x2 accumulators each.
+// EMU: every fourth pair's exponentials run on the FMA pipe (exp2_fma2), for
+// d = 64, where the MUFU unit and not the tensor core bounds the forward.
+template <bool EMU>
 __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], float sl2,
                                                   float m, uint32_t s_tm, float& l, float& lr) {
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -116,8 +119,13 @@ __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], f
                                       sl2x2, negm2);
             float x0, x1;
             f2_unpack(x2, x0, x1);
-            const float p0 = ex2_approx(x0);
-            const float p1 = ex2_approx(x1);
+            float p0, p1;
+            if (EMU && (e & 3) == 3) {
+                exp2_fma2(x0, x1, p0, p1);
+            } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+            }
             sum2[e & 1] = fadd2(sum2[e & 1], f2_pack(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
             rsum2[e & 1] = fadd2(rsum2[e & 1], f2_pack(__uint_as_float(pk[e] << 16),
@@ -466,7 +474,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             m = m_new;
-            softmax_block_exp(sr, sl2e, m, s_tm, l, lr);
+            softmax_block_exp<D == 64>(sr, sl2e, m, s_tm, l, lr);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_ready[t]);

@@ -392,6 +392,45 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
 }
 
 
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 2^x for two lanes on the FMA pipes instead of the MUFU unit (which the
+// softmax otherwise saturates).  Valid for x <= 127:
+//   * x is clamped to >= -126 (results below 2^-126 are flushed towards 0);
+//   * n = rint(x) by adding and removing the 1.5*2^23 shifter, f = x - n,
+//     f in [-1/2, 1/2] (Cody-Waite style range reduction);
+//   * 2^f ~= 1 + f*(A1 + f*(A2 + f*A3)), the degree-3 polynomial with its
+//     constant term fixed at 1 that minimises the maximum relative error on
+//     [-1/2, 1/2] (Remez exchange, exp2_poly_fit.py beside this file):
+//     relative error <= 4.4e-4, an order below the bf16 rounding the result
+//     undergoes before the PV product; integer x come out exact;
+//   * 2^x = 2^f with n added to its exponent field (the low mantissa bits of
+//     x + 1.5*2^23 hold n).
+constexpr float kExp2A1 = 0.6957668f;
+constexpr float kExp2A2 = 0.24203052f;
+constexpr float kExp2A3 = 0.04169875f;
+
+__device__ __forceinline__ void exp2_fma2(float x0, float x1, float& y0, float& y1) {
+    x0 = fmaxf(x0, -126.0f);
+    x1 = fmaxf(x1, -126.0f);
+    const uint64_t shifter = f2_pack(12582912.0f, 12582912.0f);
+    const uint64_t x = f2_pack(x0, x1);
+    const uint64_t t = fadd2(x, shifter);
+    const uint64_t f = fsub2(x, fsub2(t, shifter));
+    uint64_t p = ffma2(f, f2_pack(kExp2A3, kExp2A3), f2_pack(kExp2A2, kExp2A2));
+    p = ffma2(p, f, f2_pack(kExp2A1, kExp2A1));
+    p = ffma2(p, f, f2_pack(1.0f, 1.0f));
+    float t0, t1, p0, p1;
+    f2_unpack(t, t0, t1);
+    f2_unpack(p, p0, p1);
+    y0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
+    y1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
+}
+
 // Packs two floats to bf16x2 (round to nearest even): `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
