@@ -336,49 +336,67 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
             const uint32_t st_base = smem_u32(smem + T::ST_OFF);
             const uint32_t ds_base = smem_u32(smem + T::DS_OFF);
             // S^T_b = K Q^T and dP^T_b = V dO^T: M=128 keys, N=64 queries, K=D.
+            // Base descriptors of the fixed tiles; K steps add byte offsets.
+            const uint64_t dk0 = sdesc_sw128(k_base, 16, 1024);
+            const uint64_t dv0 = sdesc_sw128(v_base, 16, 1024);
+            const uint64_t dkt0 = sdesc_sw128(k_base, T::KV_CHUNK, 1024);
             auto mma_sdp = [&](int k, int b) {
                 const uint32_t sq = st_base + (k % T::NSTAGE) * T::STAGE_BYTES;
+                const uint64_t dq0 = sdesc_sw128(sq, 16, 1024);
+                const uint64_t ddo0 = sdesc_sw128(sq + T::Q_TILE, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t offk = (kk >> 2) * T::KV_CHUNK + (kk & 3) * 32;
                     const uint32_t offq = (kk >> 2) * T::Q_CHUNK + (kk & 3) * 32;
-                    umma_ss(tmem + 128u * b, sdesc_sw128(k_base + offk, 16, 1024),
-                            sdesc_sw128(sq + offq, 16, 1024), T::IDESC_SDP, kk > 0 ? 1u : 0u);
+                    if (kk == 0)
+                        umma_ss_c<false>(tmem + 128u * b, dk0, dq0, T::IDESC_SDP);
+                    else
+                        umma_ss_c<true>(tmem + 128u * b, sdesc_add(dk0, offk),
+                                        sdesc_add(dq0, offq), T::IDESC_SDP);
                 }
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t offk = (kk >> 2) * T::KV_CHUNK + (kk & 3) * 32;
                     const uint32_t offq = (kk >> 2) * T::Q_CHUNK + (kk & 3) * 32;
-                    umma_ss(tmem + 128u * b + 64u, sdesc_sw128(v_base + offk, 16, 1024),
-                            sdesc_sw128(sq + T::Q_TILE + offq, 16, 1024), T::IDESC_SDP,
-                            kk > 0 ? 1u : 0u);
+                    if (kk == 0)
+                        umma_ss_c<false>(tmem + 128u * b + 64u, dv0, ddo0, T::IDESC_SDP);
+                    else
+                        umma_ss_c<true>(tmem + 128u * b + 64u, sdesc_add(dv0, offk),
+                                        sdesc_add(ddo0, offq), T::IDESC_SDP);
                 }
             };
             // dV += P^T dO and dK += dS^T Q: M=128 keys, N=D, K=64 queries;
             // A (P^T or dS^T) from TMEM, B (dO or Q) MN-major from the stage.
             auto mma_dkdv = [&](int k, int b) {
                 const uint32_t sq = st_base + (k % T::NSTAGE) * T::STAGE_BYTES;
+                const uint64_t bq0 = sdesc_sw128(sq, T::Q_CHUNK, 1024);
+                const uint64_t bdo0 = sdesc_sw128(sq + T::Q_TILE, T::Q_CHUNK, 1024);
 #pragma unroll
                 for (int kk = 0; kk < T::BM / 16; ++kk) {
-                    const uint32_t acc = (k > 0 || kk > 0) ? 1u : 0u;
                     const uint32_t a_col = 128u * b + 32u * (kk >> 1) + 8u * (kk & 1);
-                    umma_ts(tmem + T::DV_COL, tmem + a_col,
-                            sdesc_sw128(sq + T::Q_TILE + kk * 2048, T::Q_CHUNK, 1024), T::IDESC_ACC,
-                            acc);
-                    umma_ts(tmem + T::DK_COL, tmem + a_col + 16u,
-                            sdesc_sw128(sq + kk * 2048, T::Q_CHUNK, 1024), T::IDESC_ACC, acc);
+                    if (kk == 0) {  // the first query block overwrites, later ones accumulate
+                        umma_ts(tmem + T::DV_COL, tmem + a_col, bdo0, T::IDESC_ACC, k > 0);
+                        umma_ts(tmem + T::DK_COL, tmem + a_col + 16u, bq0, T::IDESC_ACC, k > 0);
+                    } else {
+                        umma_ts_c<true>(tmem + T::DV_COL, tmem + a_col, sdesc_add(bdo0, kk * 2048),
+                                        T::IDESC_ACC);
+                        umma_ts_c<true>(tmem + T::DK_COL, tmem + a_col + 16u,
+                                        sdesc_add(bq0, kk * 2048), T::IDESC_ACC);
+                    }
                 }
             };
             // dQ^T = K^T dS^T: M=128 (head dim; rows >= D unused), N=64
             // queries, K=128 keys; both operands MN-major in shared memory.
             auto mma_dq = [&](int k, int b1) {
-                const uint32_t ds = ds_base + (k & 1) * T::DS_TILE;
+                const uint64_t dds0 = sdesc_sw128(ds_base + (k & 1) * T::DS_TILE, T::DS_TILE, 1024);
 #pragma unroll
-                for (int kk = 0; kk < T::BN / 16; ++kk)
-                    umma_ss(tmem + 128u * b1 + 64u,
-                            sdesc_sw128(k_base + kk * 2048, T::KV_CHUNK, 1024),
-                            sdesc_sw128(ds + kk * 2048, T::DS_TILE, 1024), T::IDESC_DQ,
-                            kk > 0 ? 1u : 0u);
+                for (int kk = 0; kk < T::BN / 16; ++kk) {
+                    if (kk == 0)
+                        umma_ss_c<false>(tmem + 128u * b1 + 64u, dkt0, dds0, T::IDESC_DQ);
+                    else
+                        umma_ss_c<true>(tmem + 128u * b1 + 64u, sdesc_add(dkt0, kk * 2048),
+                                        sdesc_add(dds0, kk * 2048), T::IDESC_DQ);
+                }
             };
             bool ok = mbar_wait(bar_kv, 0, st);
             for (int k = 0; k < 2 && k < n && ok; ++k) {

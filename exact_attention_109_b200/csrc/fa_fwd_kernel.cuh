@@ -74,8 +74,8 @@ struct FwdTraits {
     static constexpr int LOAD_WARP = 9;
     static constexpr int BIAS_WARP = 10;
     // Register split: softmax warpgroups grow, the MMA/TMA warpgroup shrinks.
-    static constexpr uint32_t REG_SOFTMAX = 216;
-    static constexpr uint32_t REG_CONTROL = 72;
+    static constexpr uint32_t REG_SOFTMAX = 208;
+    static constexpr uint32_t REG_CONTROL = 88;
     static constexpr int REG_BUDGET = 128 * (2 * REG_SOFTMAX + REG_CONTROL);
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC_S = QK8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, 0, 0);
@@ -293,25 +293,34 @@ __global__ void __launch_bounds__(384, 1)
             auto slot_par = [&](int idx) { return static_cast<uint32_t>((idx / T::NSLOT) & 1); };
             // S_t = Q_t K^T : M=128, N=128, K=D, both operands K-major;
             // each MMA consumes 32 bytes of every row (16 bf16 or 32 e4m3).
+            // Descriptors: one base per tile, K steps add byte offsets.
             auto mma_s = [&](int t, uint32_t k_addr) {
+                const uint64_t dq0 = sdesc_sw128(q_base + t * T::QK_TILE_BYTES, 16, 1024);
+                const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
 #pragma unroll
                 for (int k = 0; k < T::S_KSTEPS; ++k) {
                     const uint32_t off = (k >> 2) * T::CHUNK_BYTES + (k & 3) * 32;
-                    const uint64_t a = sdesc_sw128(q_base + t * T::QK_TILE_BYTES + off, 16, 1024);
-                    const uint64_t b = sdesc_sw128(k_addr + off, 16, 1024);
+                    const uint64_t a = sdesc_add(dq0, off);
+                    const uint64_t b = sdesc_add(dk0, off);
                     if constexpr (QK8)
                         umma_ss_f8(tmem + 128u * t, a, b, T::IDESC_S, k > 0 ? 1u : 0u);
+                    else if (k == 0)
+                        umma_ss_c<false>(tmem + 128u * t, a, b, T::IDESC_S);
                     else
-                        umma_ss(tmem + 128u * t, a, b, T::IDESC_S, k > 0 ? 1u : 0u);
+                        umma_ss_c<true>(tmem + 128u * t, a, b, T::IDESC_S);
                 }
             };
             // O_t += P_t V : M=128, N=D, K=128; P from TMEM, V MN-major.
             auto mma_pv = [&](int t, uint32_t v_addr, bool accumulate) {
+                const uint64_t dv0 = sdesc_sw128(v_addr, T::CHUNK_BYTES, 1024);
 #pragma unroll
                 for (int k = 0; k < T::BN / 16; ++k) {
-                    const uint64_t b = sdesc_sw128(v_addr + k * 2048, T::CHUNK_BYTES, 1024);
-                    umma_ts(tmem + 256u + D * t, tmem + 128u * t + 8u * k, b, T::IDESC_PV,
-                            (accumulate || k > 0) ? 1u : 0u);
+                    if (k == 0)
+                        umma_ts(tmem + 256u + D * t, tmem + 128u * t, dv0, T::IDESC_PV,
+                                accumulate ? 1u : 0u);
+                    else
+                        umma_ts_c<true>(tmem + 256u + D * t, tmem + 128u * t + 8u * k,
+                                        sdesc_add(dv0, k * 2048), T::IDESC_PV);
                 }
             };
             bool ok = mbar_wait(bar_q, 0, st) && mbar_wait(&full[0], 0, st);
