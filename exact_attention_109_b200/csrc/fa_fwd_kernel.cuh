@@ -98,16 +98,21 @@ struct FwdParams {
 
 // One softmax row over a 128-key block: p = exp2(s * scale*log2(e) - m) in
 // pairs (f32x2 FFMA for the argument), packed to bf16 and written over the
-// first 64 TMEM columns of S; returns the fp32 sum of p (for the LSE) and of
-// the bf16-rounded p (for normalising O) through two f32x2 accumulators each.
-// EMU: every fourth pair's exponentials run on the FMA pipe (exp2_fma2), for
-// d = 64, where the MUFU unit and not the tensor core bounds the forward.
-template <bool EMU>
+// first 64 TMEM columns of S; adds the fp32 sum of p (for the LSE) to l and
+// the sum of the bf16-rounded p (for normalising O) to lr.  The rounded
+// weights are summed straight from the packed bf16 pairs with mixed-precision
+// adds (exact widening, fp32 sum).  Every fourth pair's exponentials run on
+// the FMA pipe (exp2_fma2) instead of the MUFU unit: one MUFU ex2 per score
+// against 4*d tensor FLOP per score puts the two units at about the same time
+// per block at d = 128 and MUFU at twice the tensor time at d = 64, so moving
+// a quarter of the exponentials to the FMA pipe shortens the softmax that
+// each tile's next MMAs wait for.
 __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], float sl2,
                                                   float m, uint32_t s_tm, float& l, float& lr) {
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     const uint64_t negm2 = f2_pack(-m, -m);
-    uint64_t sum2[2] = {0ull, 0ull}, rsum2[2] = {0ull, 0ull};
+    uint64_t sum2[2] = {0ull, 0ull};
+    float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
@@ -120,7 +125,7 @@ __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], f
             float x0, x1;
             f2_unpack(x2, x0, x1);
             float p0, p1;
-            if (EMU && (e & 3) == 3) {
+            if ((e & 3) == 3) {
                 exp2_fma2(x0, x1, p0, p1);
             } else {
                 p0 = ex2_approx(x0);
@@ -128,16 +133,14 @@ __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], f
             }
             sum2[e & 1] = fadd2(sum2[e & 1], f2_pack(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
-            rsum2[e & 1] = fadd2(rsum2[e & 1], f2_pack(__uint_as_float(pk[e] << 16),
-                                                       __uint_as_float(pk[e] & 0xffff0000u)));
+            add_bf16x2_to_f32(pk[e], rs[2 * (e & 1)], rs[2 * (e & 1) + 1]);
         }
         tmem_st32(s_tm + 32u * h, pk);
     }
-    float a0, a1, b0, b1;
+    float a0, a1;
     f2_unpack(fadd2(sum2[0], sum2[1]), a0, a1);
-    f2_unpack(fadd2(rsum2[0], rsum2[1]), b0, b1);
     l += a0 + a1;
-    lr += b0 + b1;
+    lr += (rs[0] + rs[1]) + (rs[2] + rs[3]);
 }
 
 template <int D, bool CAUSAL, bool QK8 = false, bool BIAS = false>
@@ -483,7 +486,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             m = m_new;
-            softmax_block_exp<D == 64>(sr, sl2e, m, s_tm, l, lr);
+            softmax_block_exp(sr, sl2e, m, s_tm, l, lr);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_ready[t]);

@@ -407,6 +407,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
     return y;
 }
 
+// acc + lo and acc + hi, where lo and hi are the two bf16 halves of `pk`,
+// each widened exactly and added in fp32 (sm_100 mixed-precision add).
+__device__ __forceinline__ void add_bf16x2_to_f32(uint32_t pk, float& acc_lo, float& acc_hi) {
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi) : "r"(pk));
+}
+
 // Two-lane fp32 vectors in one 64-bit register pair (sm_100 f32x2 ops).
 __device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
     uint64_t r;
