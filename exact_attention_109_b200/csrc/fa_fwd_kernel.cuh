@@ -65,8 +65,8 @@ struct FwdTraits {
     static constexpr int BIAS_OFF = OST_OFF + (QK8 ? TILES * TILE_BYTES : 0);
     static constexpr int BAR_OFF = BIAS_OFF + (BIAS ? TILES * BIAS_TILE : 0);
     // q, full[NSLOT], empty[NSLOT], s_full[2], p_ready[2], o_final[2],
-    // mma_done, bias_full[2], bias_empty[2]
-    static constexpr int NBAR = 1 + 2 * NSLOT + 2 + 2 + 2 + 1 + 4;
+    // mma_done, bias_full[2], bias_empty[2], p_half[2]
+    static constexpr int NBAR = 1 + 2 * NSLOT + 2 + 2 + 2 + 1 + 4 + 2;
     static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
     static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + alignment slack
     static constexpr int NUM_THREADS = 384;  // 3 warpgroups; warps 10-11 idle
@@ -81,6 +81,10 @@ struct FwdTraits {
     static constexpr uint32_t IDESC_S = QK8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, 0, 0);
     static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
     static constexpr float TAU = 8.0f;  // deferred-rescale threshold (log2 units)
+    // The softmax signals P per 64-key half and the PV MMA starts on the
+    // first half early.  At d = 64 (softmax-bound) that gains; at d = 128
+    // the extra TMEM-store wait in the middle of the softmax costs more.
+    static constexpr bool PSPLIT = (D == 64);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -106,9 +110,13 @@ struct FwdParams {
 // against 4*d tensor FLOP per score puts the two units at about the same time
 // per block at d = 128 and MUFU at twice the tensor time at d = 64, so moving
 // a quarter of the exponentials to the FMA pipe shortens the softmax that
-// each tile's next MMAs wait for.
+// each tile's next MMAs wait for.  PSPLIT: the first 64 keys' P is made
+// visible to the tensor core and `half_bar` arrived on before the second half
+// is computed.
+template <bool PSPLIT>
 __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], float sl2,
-                                                  float m, uint32_t s_tm, float& l, float& lr) {
+                                                  float m, uint32_t s_tm, float& l, float& lr,
+                                                  uint64_t* half_bar) {
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     const uint64_t negm2 = f2_pack(-m, -m);
     uint64_t sum2[2] = {0ull, 0ull};
@@ -136,6 +144,11 @@ __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], f
             add_bf16x2_to_f32(pk[e], rs[2 * (e & 1)], rs[2 * (e & 1) + 1]);
         }
         tmem_st32(s_tm + 32u * h, pk);
+        if (PSPLIT && h == 0) {
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(half_bar);
+        }
     }
     float a0, a1;
     f2_unpack(fadd2(sum2[0], sum2[1]), a0, a1);
@@ -162,6 +175,7 @@ __global__ void __launch_bounds__(384, 1)
     uint64_t* mma_done = o_final + 2;
     uint64_t* bias_full = mma_done + 1;
     uint64_t* bias_empty = bias_full + 2;
+    uint64_t* p_half = bias_empty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + T::MISC_OFF);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + T::MISC_OFF + 4);
 
@@ -197,6 +211,7 @@ __global__ void __launch_bounds__(384, 1)
             mbar_init(&o_final[t], 1);
             mbar_init(&bias_full[t], 1);
             mbar_init(&bias_empty[t], 128);
+            mbar_init(&p_half[t], 128);
         }
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -314,10 +329,11 @@ __global__ void __launch_bounds__(384, 1)
                 }
             };
             // O_t += P_t V : M=128, N=D, K=128; P from TMEM, V MN-major.
-            auto mma_pv = [&](int t, uint32_t v_addr, bool accumulate) {
+            // K steps [k0, k1) of O_t += P_t V (16 keys each).
+            auto mma_pv = [&](int t, uint32_t v_addr, bool accumulate, int k0, int k1) {
                 const uint64_t dv0 = sdesc_sw128(v_addr, T::CHUNK_BYTES, 1024);
 #pragma unroll
-                for (int k = 0; k < T::BN / 16; ++k) {
+                for (int k = k0; k < k1; ++k) {
                     if (k == 0)
                         umma_ts(tmem + 256u + D * t, tmem + 128u * t, dv0, T::IDESC_PV,
                                 accumulate ? 1u : 0u);
@@ -325,6 +341,23 @@ __global__ void __launch_bounds__(384, 1)
                         umma_ts_c<true>(tmem + 256u + D * t, tmem + 128u * t + 8u * k,
                                         sdesc_add(dv0, k * 2048), T::IDESC_PV);
                 }
+            };
+            // PV of tile t for the block whose P has phase `par`: in two
+            // 64-key halves when the softmax signals them separately.
+            auto pv_tile = [&](int t, uint32_t v_addr, bool acc, uint32_t par) -> bool {
+                if constexpr (T::PSPLIT) {
+                    if (!mbar_wait(&p_half[t], par, st)) return false;
+                    tc_fence_after();
+                    mma_pv(t, v_addr, acc, 0, T::BN / 32);
+                    if (!mbar_wait(&p_ready[t], par, st)) return false;
+                    tc_fence_after();
+                    mma_pv(t, v_addr, true, T::BN / 32, T::BN / 16);
+                } else {
+                    if (!mbar_wait(&p_ready[t], par, st)) return false;
+                    tc_fence_after();
+                    mma_pv(t, v_addr, acc, 0, T::BN / 16);
+                }
+                return true;
             };
             bool ok = mbar_wait(bar_q, 0, st) && mbar_wait(&full[0], 0, st);
             if (ok) {
@@ -342,18 +375,14 @@ __global__ void __launch_bounds__(384, 1)
                 if (!ok) break;
                 tc_fence_after();
                 if (j - 1 < n0) {
-                    if (!(ok = mbar_wait(&p_ready[0], (j - 1) & 1, st))) break;
-                    tc_fence_after();
-                    mma_pv(0, slot_addr(iv), j - 1 > 0);
+                    if (!(ok = pv_tile(0, slot_addr(iv), j - 1 > 0, (j - 1) & 1))) break;
                     if (j - 1 == n0 - 1) umma_commit(&o_final[0]);
                 }
                 if (j < n0) {
                     mma_s(0, slot_addr(ik));
                     umma_commit(&s_full[0]);
                 }
-                if (!(ok = mbar_wait(&p_ready[1], (j - 1) & 1, st))) break;
-                tc_fence_after();
-                mma_pv(1, slot_addr(iv), j - 1 > 0);
+                if (!(ok = pv_tile(1, slot_addr(iv), j - 1 > 0, (j - 1) & 1))) break;
                 umma_commit(&empty[iv % T::NSLOT]);
                 mma_s(1, slot_addr(ik));
                 umma_commit(&s_full[1]);
@@ -363,17 +392,11 @@ __global__ void __launch_bounds__(384, 1)
                 const int jl = n1 - 1, iv = 2 * n1 - 1;
                 ok = mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st);
                 if (ok && jl < n0) {
-                    ok = mbar_wait(&p_ready[0], jl & 1, st);
-                    if (ok) {
-                        tc_fence_after();
-                        mma_pv(0, slot_addr(iv), jl > 0);
-                        umma_commit(&o_final[0]);
-                    }
+                    ok = pv_tile(0, slot_addr(iv), jl > 0, jl & 1);
+                    if (ok) umma_commit(&o_final[0]);
                 }
-                if (ok) ok = mbar_wait(&p_ready[1], jl & 1, st);
+                if (ok) ok = pv_tile(1, slot_addr(iv), jl > 0, jl & 1);
                 if (ok) {
-                    tc_fence_after();
-                    mma_pv(1, slot_addr(iv), jl > 0);
                     umma_commit(&o_final[1]);
                     umma_commit(&empty[iv % T::NSLOT]);
                 }
@@ -486,7 +509,7 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             m = m_new;
-            softmax_block_exp(sr, sl2e, m, s_tm, l, lr);
+            softmax_block_exp<T::PSPLIT>(sr, sl2e, m, s_tm, l, lr, &p_half[t]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_ready[t]);
