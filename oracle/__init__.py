@@ -49,7 +49,7 @@ def open_library(path: str):
     lib.ref_bwd.restype = i
     lib.ref_fwd_rows.argtypes = [_D, _D, _D, i, i, i, d, _LL, i, _D, _D]
     lib.ref_fwd_rows.restype = i
-    lib.ref_head_stats.argtypes = [_D, _D, _D, _D, i, i, i, d, _D, _D]
+    lib.ref_head_stats.argtypes = [_D, _D, _D, _D, i, i, i, d, i, _D, _D]
     lib.ref_head_stats.restype = i
     lib.ref_dq_rows.argtypes = [_D, _D, _D, _D, i, i, i, d, _LL, i, _D]
     lib.ref_dq_rows.restype = i
@@ -136,15 +136,19 @@ def ref_fwd_rows(q, k, v, rows, causal: bool, scale: float, lib=None):
     return o, lse
 
 
-def ref_head_stats(q, k, v, dO, causal: bool, scale: float, lib=None):
-    """LSE_i and D_i for every query row of one head ([N,d] inputs)."""
+def ref_head_stats(q, k, v, dO, causal: bool, scale: float, lib=None, first: int = 0):
+    """LSE_i and D_i for the query rows i >= ``first`` of one head ([N,d]
+    inputs); earlier rows are NaN.  Under the causal mask these are all the
+    statistics that dK/dV rows j >= ``first`` depend on."""
     lib = lib or _load()
     q, k, v, dO = _f64(q), _f64(k), _f64(v), _f64(dO)
     N, d = q.shape
-    lse = np.empty(N, dtype=np.float64)
-    D = np.empty(N, dtype=np.float64)
+    if not 0 <= first <= N:
+        raise ValueError("first must lie in [0, N]")
+    lse = np.full(N, np.nan, dtype=np.float64)
+    D = np.full(N, np.nan, dtype=np.float64)
     rc = lib.ref_head_stats(_p(q), _p(k), _p(v), _p(dO), N, d,
-                            int(bool(causal)), float(scale), _p(lse), _p(D))
+                            int(bool(causal)), float(scale), int(first), _p(lse), _p(D))
     if rc:
         raise MemoryError("oracle: allocation failed")
     return lse, D

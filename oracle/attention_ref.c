@@ -210,18 +210,21 @@ int ref_fwd_rows(const double *q, const double *k, const double *v, int N,
 
 /*
  * Per-row softmax statistics of one head: LSE_i and D_i = sum_j P_ij dP_ij for
- * every query row.  Costs O(N^2 d); used to sample dK/dV rows at large N.
+ * the query rows i in [first, N) (rows before `first` are left untouched).
+ * Costs O((N - first) N d); used to sample dK/dV rows at large N.  Under the
+ * causal mask, key row j only meets query rows i >= j, so the statistics of
+ * the rows from `first` on are all that dK/dV rows j >= first need.
  */
 int ref_head_stats(const double *q, const double *k, const double *v,
                    const double *dO, int N, int d, int causal, double scale,
-                   double *lse, double *D) {
+                   int first, double *lse, double *D) {
     int failed = 0;
 #pragma omp parallel reduction(| : failed)
     {
         double *p = (double *)malloc(sizeof(double) * (size_t)N);
         if (!p) failed = 1;
 #pragma omp for schedule(dynamic, 16)
-        for (int i = 0; i < N; ++i) {
+        for (int i = first; i < N; ++i) {
             if (!p) continue;
             const int n = row_extent(i, N, causal);
             lse[i] = forward_row(q + (size_t)i * d, k, v, n, d, scale, p, NULL);

@@ -171,3 +171,30 @@ def check_backward_sampled(host, dq, dk, dv, causal, scale, heads, rows_per_head
     for name in ("dq", "dk", "dv"):
         assert res[name + "_excess"] <= TOL_GRAD_MAX, res
     return res
+
+
+def check_backward_causal_tail(host, dq, dk, dv, scale, heads, rows_per_head, tail, seed=0):
+    """Causal mask at large N: exact oracle dQ for sampled query rows anywhere
+    in each listed head, and exact dK/dV for sampled key rows among the last
+    ``tail`` keys, which only meet the last ``tail`` queries (so the oracle
+    needs the softmax statistics of those rows alone)."""
+    B, H, N, d = host["q"].shape
+    first = N - tail
+    rng = np.random.default_rng(seed)
+    flat = {x: host[x].reshape(B * H, N, d) for x in ("q", "k", "v", "dO")}
+    res = {f"{n}_{m}": 0.0 for n in ("dq", "dk", "dv") for m in ("excess", "max")}
+    for bh in heads:
+        q, k, v, dO = (to_f64(flat[x][bh]) for x in ("q", "k", "v", "dO"))
+        q_rows = sample_rows(N, rows_per_head, rng)
+        k_rows = first + sample_rows(tail, rows_per_head, rng)
+        lse_h, D_h = oracle.ref_head_stats(q, k, v, dO, True, scale, first=first)
+        rdq = oracle.ref_dq_rows(q, k, v, dO, q_rows, True, scale)
+        rdk, rdv = oracle.ref_dkdv_rows(q, k, v, dO, lse_h, D_h, k_rows, True, scale)
+        for name, got, ref, rows in (("dq", dq, rdq, q_rows), ("dk", dk, rdk, k_rows),
+                                     ("dv", dv, rdv, k_rows)):
+            g = to_f64(got.reshape(B * H, N, d)[bh].cpu()[torch.from_numpy(rows)])
+            res[name + "_excess"] = max(res[name + "_excess"], max_excess(g, ref))
+            res[name + "_max"] = max(res[name + "_max"], max_abs(g, ref))
+    for name in ("dq", "dk", "dv"):
+        assert res[name + "_excess"] <= TOL_GRAD_MAX, res
+    return res

@@ -5,8 +5,8 @@ import torch
 
 import exact_attention_109_b200 as fa
 from exact_attention_109_b200.inputs import default_scale
-from parity_util import (check_backward_heads, check_backward_sampled,
-                         gpu_inputs, run_backward, run_forward)
+from parity_util import (check_backward_causal_tail, check_backward_heads,
+                         check_backward_sampled, gpu_inputs, run_backward, run_forward)
 
 pytestmark = pytest.mark.gpu
 
@@ -51,6 +51,20 @@ def test_sweep_sampled(N, d, causal):
     B, H = 16384 // N, 2048 // d
     host, dq, dk, dv, scale = _fwd_bwd(B, H, N, d, causal, seed=2)
     check_backward_sampled(host, dq, dk, dv, causal, scale, [B * H - 1], 32)
+
+
+def test_bench_workload_sampled():
+    """The benchmark's step at full size: B=2 H=16 N=8192 d=128 causal, the
+    same seeded inputs, sampled rows of the first and last heads."""
+    host, dq, dk, dv, scale = _fwd_bwd(2, 16, 8192, 128, True, seed=2)
+    check_backward_sampled(host, dq, dk, dv, True, scale, [0, 31], 32)
+
+
+def test_long_sequence_sampled():
+    """B=1 H=16 N=65536 d=128 causal: dQ rows anywhere in two heads, dK/dV
+    rows among the last 512 keys."""
+    host, dq, dk, dv, scale = _fwd_bwd(1, 16, 65536, 128, True, seed=3)
+    check_backward_causal_tail(host, dq, dk, dv, scale, [0, 15], 16, 512)
 
 
 def test_row_scaled_gpt_layer():

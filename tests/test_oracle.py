@@ -379,6 +379,28 @@ def test_online_softmax_matches_and_blockwise_normalisation_does_not():
         assert np.max(np.abs(Obad - o[0, 0])) > 1e-2
 
 
+def test_tail_head_stats_serve_causal_tail_key_rows():
+    """Statistics of the rows from `first` on equal the full ones there (NaN
+    before), and under the causal mask they give the full dK/dV of the key
+    rows from `first` on, since those keys only meet the later queries."""
+    q, k, v, dO = rng_inputs(23, 1, 1, 150, 8)
+    first = 97
+    lse_f, D_f = oracle.ref_head_stats(q[0, 0], k[0, 0], v[0, 0], dO[0, 0], True, 0.3)
+    lse_t, D_t = oracle.ref_head_stats(q[0, 0], k[0, 0], v[0, 0], dO[0, 0], True, 0.3,
+                                       first=first)
+    assert np.all(np.isnan(lse_t[:first])) and np.all(np.isnan(D_t[:first]))
+    np.testing.assert_array_equal(lse_t[first:], lse_f[first:])
+    np.testing.assert_array_equal(D_t[first:], D_f[first:])
+    _, dk, dv, _ = oracle.ref_bwd(q, k, v, dO, True, 0.3)
+    rows = np.array([first, 120, 149])
+    dk_r, dv_r = oracle.ref_dkdv_rows(q[0, 0], k[0, 0], v[0, 0], dO[0, 0], lse_t, D_t,
+                                      rows, True, 0.3)
+    np.testing.assert_allclose(dk_r, dk[0, 0, rows], atol=1e-13)
+    np.testing.assert_allclose(dv_r, dv[0, 0, rows], atol=1e-13)
+    with pytest.raises(ValueError):
+        oracle.ref_head_stats(q[0, 0], k[0, 0], v[0, 0], dO[0, 0], True, 0.3, first=151)
+
+
 def test_sampled_rows_match_full_tensors():
     q, k, v, dO = rng_inputs(19, 1, 1, 150, 8)
     rows = np.array([0, 1, 63, 64, 127, 128, 149])
