@@ -426,6 +426,9 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
                     if (!ok) break;
                     tc_fence_after();
                     mma_sdp(k + 2, b);
+                    // This commit completes only after dQ^T(k) above has read
+                    // dS^T buffer k & 1, which block k+2's P/dS warps rewrite
+                    // once they see it: keep S/dP(k+2) after dQ^T(k).
                     umma_commit(&sdp_full[b]);
                 }
             }
