@@ -53,6 +53,19 @@ def attention_inputs(B: int, H: int, N: int, d: int, seed: int,
     return out
 
 
+def attention_inputs_device(B: int, H: int, N: int, d: int, seed: int,
+                            device="cuda"):
+    """q, k, v, dO of shape [B,H,N,d], "normal" recipe, drawn directly on the
+    device by a seeded ``torch.Generator`` of that device (in the order q, k,
+    v, dO) -- for shapes whose host-side generation and transfer would take
+    minutes.  The bits differ from ``attention_inputs`` with the same seed;
+    a caller that checks a slice against the oracle copies that slice back."""
+    gen = torch.Generator(device).manual_seed(int(seed))
+    shape = (B, H, N, d)
+    return {name: torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+            .to(torch.bfloat16) for name in ("q", "k", "v", "dO")}
+
+
 def decode_inputs(B: int, H: int, Nq: int, Nk: int, d: int, seed: int,
                   dist: str = "normal"):
     """CPU bf16 q [B,H,Nq,d] and k, v [B,H,Nk,d] for decoding (Nq query rows
