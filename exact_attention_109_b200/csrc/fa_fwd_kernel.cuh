@@ -198,6 +198,13 @@ __global__ void __launch_bounds__(384, 1)
     const int n_kv = (N + T::BN - 1) / T::BN;
     const int n0 = CAUSAL ? min(n_kv, 2 * qp + 1) : n_kv;  // key blocks of tile 0
     const int n1 = CAUSAL ? min(n_kv, 2 * qp + 2) : n_kv;  // key blocks of tile 1
+    // Causal: the key blocks are walked from the diagonal down, so tile 1's
+    // extra block (its diagonal, hidden from tile 0) comes first, while tile
+    // 0's first scores are computed, and both tiles end on block 0 together
+    // (in ascending order tile 1's last block would run with no partner).
+    // Iteration i visits key block kv_block(i); tile 0 joins at i = off0.
+    const int off0 = CAUSAL ? n1 - n0 : 0;
+    auto kv_block = [&](int i) { return CAUSAL ? n1 - 1 - i : i; };
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q, 1);
@@ -260,7 +267,7 @@ __global__ void __launch_bounds__(384, 1)
                     const int ccols = h ? 64 : T::QK_CHUNK_COLS;
                     for (int c = 0; c < nch; ++c)
                         tma_load_3d(dst + c * T::CHUNK_BYTES, h ? &tmV : &tmK, &full[slot],
-                                    c * ccols, j * T::BN, bh);
+                                    c * ccols, kv_block(j) * T::BN, bh);
                     ++issued;
                 }
             }
@@ -282,8 +289,10 @@ __global__ void __launch_bounds__(384, 1)
             bool ok = true;
             for (int j = 0; j < n1 && ok; ++j) {
                 for (int t = 0; t < 2; ++t) {
-                    if (j >= (t ? n1 : n0)) continue;
-                    if (j > 0 && !mbar_wait(&bias_empty[t], (j - 1) & 1, st)) {
+                    if (t == 0 && (j < off0 || j - off0 >= n0)) continue;
+                    // the previous tile of this query tile must have been read
+                    if (issued[t] > 0 &&
+                        !mbar_wait(&bias_empty[t], (issued[t] - 1) & 1, st)) {
                         ok = false;
                         break;
                     }
@@ -291,7 +300,7 @@ __global__ void __launch_bounds__(384, 1)
                     uint8_t* dst = smem + T::BIAS_OFF + t * T::BIAS_TILE;
                     for (int c = 0; c < 2; ++c)
                         tma_load_3d(dst + c * T::CHUNK_BYTES, &tmB, &bias_full[t],
-                                    j * T::BN + 64 * c, q0 + 128 * t, bz);
+                                    kv_block(j) * T::BN + 64 * c, q0 + 128 * t, bz);
                     ++issued[t];
                 }
             }
@@ -359,26 +368,32 @@ __global__ void __launch_bounds__(384, 1)
                 }
                 return true;
             };
+            // Tile 0 takes part in iterations [off0, off0 + n0); its own block
+            // count (for its barrier phases) is i - off0.
+            auto act0 = [&](int i) { return i >= off0 && i - off0 < n0; };
             bool ok = mbar_wait(bar_q, 0, st) && mbar_wait(&full[0], 0, st);
             if (ok) {
                 tc_fence_after();
-                mma_s(0, slot_addr(0));
-                umma_commit(&s_full[0]);
+                if (act0(0)) {
+                    mma_s(0, slot_addr(0));
+                    umma_commit(&s_full[0]);
+                }
                 mma_s(1, slot_addr(0));
                 umma_commit(&s_full[1]);
                 umma_commit(&empty[0]);
             }
             for (int j = 1; j < n1 && ok; ++j) {
-                const int ik = 2 * j, iv = 2 * j - 1;  // K_j and V_{j-1}
+                const int ik = 2 * j, iv = 2 * j - 1;  // K of iteration j, V of j-1
                 ok = mbar_wait(&full[ik % T::NSLOT], slot_par(ik), st) &&
                      mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st);
                 if (!ok) break;
                 tc_fence_after();
-                if (j - 1 < n0) {
-                    if (!(ok = pv_tile(0, slot_addr(iv), j - 1 > 0, (j - 1) & 1))) break;
-                    if (j - 1 == n0 - 1) umma_commit(&o_final[0]);
+                if (act0(j - 1)) {
+                    const int l0 = j - 1 - off0;
+                    if (!(ok = pv_tile(0, slot_addr(iv), l0 > 0, l0 & 1))) break;
+                    if (l0 == n0 - 1) umma_commit(&o_final[0]);
                 }
-                if (j < n0) {
+                if (act0(j)) {
                     mma_s(0, slot_addr(ik));
                     umma_commit(&s_full[0]);
                 }
@@ -391,8 +406,9 @@ __global__ void __launch_bounds__(384, 1)
             if (ok) {
                 const int jl = n1 - 1, iv = 2 * n1 - 1;
                 ok = mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st);
-                if (ok && jl < n0) {
-                    ok = pv_tile(0, slot_addr(iv), jl > 0, jl & 1);
+                if (ok && act0(jl)) {
+                    const int l0 = jl - off0;
+                    ok = pv_tile(0, slot_addr(iv), l0 > 0, l0 & 1);
                     if (ok) umma_commit(&o_final[0]);
                 }
                 if (ok) ok = pv_tile(1, slot_addr(iv), jl > 0, jl & 1);
@@ -465,7 +481,8 @@ __global__ void __launch_bounds__(384, 1)
             constexpr float kUnit = 1.0f;
             const float sl2e = BIAS ? kUnit : sl2;  // scale still to apply to sr
 
-            const int kv0 = j * T::BN;
+            // tile t's j-th block: key block nt-1-j when walking down
+            const int kv0 = (CAUSAL ? nt - 1 - j : j) * T::BN;
             // Only the ragged last block and (causal) the diagonal block hold
             // hidden scores; the test is uniform over the tile.
             const bool masked_block =
