@@ -223,6 +223,23 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(mma_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
+        // Q and the first key/value block are requested here, so that their
+        // latency overlaps the TMEM allocation and the block-wide sync; the
+        // producer warp continues with the second block.
+        mbar_arrive_expect_tx(bar_q, T::TILES * T::QK_TILE_BYTES);
+        for (int t = 0; t < T::TILES; ++t)
+            for (int c = 0; c < T::QK_CHUNKS; ++c)
+                tma_load_3d(smem + T::Q_OFF + t * T::QK_TILE_BYTES + c * T::CHUNK_BYTES, &tmQ,
+                            bar_q, c * T::QK_CHUNK_COLS, q0 + 128 * t, bh);
+        for (int h = 0; h < 2; ++h) {  // slots 0 and 1: K and V of iteration 0
+            mbar_arrive_expect_tx(&full[h], h ? T::TILE_BYTES : T::QK_TILE_BYTES);
+            uint8_t* dst = smem + T::KV_OFF + h * T::TILE_BYTES;
+            const int nch = h ? T::CHUNKS : T::QK_CHUNKS;
+            const int ccols = h ? 64 : T::QK_CHUNK_COLS;
+            for (int c = 0; c < nch; ++c)
+                tma_load_3d(dst + c * T::CHUNK_BYTES, h ? &tmV : &tmK, &full[h], c * ccols,
+                            kv_block(0) * T::BN, bh);
+        }
     }
     if (warp == T::MMA_WARP) {
         tmem_alloc(tmem_slot, T::TMEM_COLS);
@@ -246,13 +263,8 @@ __global__ void __launch_bounds__(384, 1)
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             bool ok = true;
-            mbar_arrive_expect_tx(bar_q, T::TILES * T::QK_TILE_BYTES);
-            for (int t = 0; t < T::TILES; ++t)
-                for (int c = 0; c < T::QK_CHUNKS; ++c)
-                    tma_load_3d(smem + T::Q_OFF + t * T::QK_TILE_BYTES + c * T::CHUNK_BYTES,
-                                &tmQ, bar_q, c * T::QK_CHUNK_COLS, q0 + 128 * t, bh);
-            int issued = 0;
-            for (int j = 0; j < n1 && ok; ++j) {
+            int issued = 2;  // Q and iteration 0's K, V were issued at set-up
+            for (int j = 1; j < n1 && ok; ++j) {
                 for (int h = 0; h < 2; ++h) {  // 0: K_j, 1: V_j
                     const int idx = 2 * j + h;
                     const int slot = idx % T::NSLOT;
