@@ -1082,6 +1082,67 @@ def bias_arm(args, w, wname):
     return 0
 
 
+def sweep_arm(args):
+    """The whole kernel sweep of the pages' benchmark on one GPU: the 16k-token
+    shapes (B*N = 16384, width 2048) for d = 64 and 128, both masks, the two
+    GPT-layer shapes (row-scaled inputs) and the N = 65536 sequence, forward
+    and backward through the public API with preallocated outputs and
+    workspace.  One JSON line per shape (not the benchmark contract's single
+    line): TFLOP/s of the forward, the backward (2.5x the forward's FLOPs)
+    and both, each the median of three CUDA-event-timed runs of ten calls."""
+    import numpy as np
+    import torch
+    import exact_attention_109_b200 as fa
+    from exact_attention_109_b200.inputs import attention_inputs, default_scale
+    torch.cuda.set_device(0)
+    cases = [(16384 // n, 32 if d == 64 else 16, n, d, c, "normal", 2)
+             for n in (512, 1024, 2048, 4096, 8192, 16384) for d in (64, 128)
+             for c in (False, True)]
+    cases += [(8, 16, 2048, 128, True, "row_scaled", 4), (2, 20, 8192, 128, True, "row_scaled", 5),
+              (1, 16, 65536, 128, True, "normal", 3)]
+    for (B, H, N, d, causal, dist, seed) in cases:
+        host = attention_inputs(B, H, N, d, seed=seed, dist=dist, with_dout=True)
+        q, k, v, dO = (host[x].cuda() for x in ("q", "k", "v", "dO"))
+        sc = default_scale(d)
+        ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
+        o = torch.empty_like(q)
+        lse = torch.empty(B, H, N, device="cuda")
+
+        def fwd():
+            fa.attention_forward(q, k, v, causal, sc, out=o, lse=lse)
+
+        def bwd():
+            fa.attention_backward(q, k, v, o, lse, dO, causal, sc, workspace=ws)
+
+        for _ in range(args.warmup):
+            fwd()
+            bwd()
+        torch.cuda.synchronize()
+        reps = 10 if N <= 16384 else 3
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        tf, tb = [], []
+        for _ in range(3):
+            ev[0].record()
+            for _ in range(reps):
+                fwd()
+            ev[1].record()
+            for _ in range(reps):
+                bwd()
+            ev[2].record()
+            torch.cuda.synchronize()
+            tf.append(ev[0].elapsed_time(ev[1]) / reps)
+            tb.append(ev[1].elapsed_time(ev[2]) / reps)
+        status = fa.fa_get_device_error()
+        if status != fa.FA_OK:
+            raise fa.FaError(status, "sweep")
+        fl = 4.0 * B * H * N * N * d * (0.5 if causal else 1.0)
+        f_ms, b_ms = float(np.median(tf)), float(np.median(tb))
+        print(json.dumps({"B": B, "H": H, "N": N, "d": d, "causal": causal, "inputs": dist,
+                          "fwd_tflops": fl / f_ms / 1e9, "bwd_tflops": 2.5 * fl / b_ms / 1e9,
+                          "fwd_bwd_tflops": 3.5 * fl / (f_ms + b_ms) / 1e9}), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1093,8 +1154,12 @@ def main():
                     + sorted(BIAS_WORKLOADS),
                     default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true",
+                    help="time the whole shape sweep (one JSON line per shape) and exit")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.sweep:
+        return sweep_arm(args)
     if args.workload in BIAS_WORKLOADS:
         if args.impl == "reference":
             return reference_arm(args, BIAS_WORKLOADS[args.workload], args.workload)
