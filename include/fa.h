@@ -32,8 +32,10 @@
  *     stream).  Work is enqueued asynchronously; no call synchronises the
  *     host except fa_get_device_error.
  *   - A status other than FA_OK means nothing was enqueued.
- *   - Supported: d in {64, 128}; N >= 1; B, H >= 1; B*H*N*d < 2^31 rows*cols
- *     per tensor index space of one head batch; scale finite and > 0.
+ *   - Supported: d in {64, 128}; N >= 1; B, H >= 1; B*H <= 2^24, N <= 2^30
+ *     and B*H*ceil(N/256) < 2^31 (grid and TMA coordinates are 32-bit);
+ *     element offsets are 64-bit, so a tensor may exceed 2^31 elements;
+ *     scale finite and > 0.
  *     causal: key j is visible to query i iff j <= i.
  *   - Device-side waits are bounded (about 2 s).  A kernel whose pipeline wait
  *     runs out records FA_ERR_TIMEOUT in the device error word and returns
