@@ -9,9 +9,15 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SOURCES = [os.path.join(HERE, "csrc", "fa_api.cu"),
            os.path.join(HERE, "csrc", "fa_noalloc.cu")]
-HEADERS = [os.path.join(HERE, "csrc", f) for f in
-           ("sm100_ptx.cuh", "fa_fwd_kernel.cuh", "fa_bwd_kernels.cuh")] + \
-          [os.path.join(ROOT, "include", "fa.h")]
+
+
+def headers():
+    """Every header the sources can include: all of csrc/*.cuh and include/*.h."""
+    out = []
+    for folder, ext in ((os.path.join(HERE, "csrc"), ".cuh"), (os.path.join(ROOT, "include"), ".h")):
+        out += sorted(os.path.join(folder, f) for f in os.listdir(folder) if f.endswith(ext))
+    return out
+
 OUT = os.path.join(HERE, "libfa_sm100.so")
 
 
@@ -26,7 +32,7 @@ def up_to_date(out: str = OUT) -> bool:
     if not os.path.exists(out):
         return False
     t = os.path.getmtime(out)
-    return all(os.path.getmtime(f) <= t for f in SOURCES + HEADERS)
+    return all(os.path.getmtime(f) <= t for f in SOURCES + headers())
 
 
 def build(force: bool = False, verbose: bool = False) -> str:

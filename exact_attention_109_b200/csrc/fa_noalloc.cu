@@ -27,12 +27,12 @@ constexpr int kMaxDevices = 64;
 // from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-struct ScratchAddress {
-    std::once_flag once;
-    void* ptr = nullptr;
-    cudaError_t err = cudaSuccess;
-};
-ScratchAddress g_scratch[kMaxDevices];
+// Device address of the array, per device; null until a lookup succeeds.
+// Only a successful lookup is cached: a failed one (for instance a first call
+// made while a stream was being captured, or a sticky error from earlier
+// work) is reported to that caller, and the next call tries again.
+std::mutex g_scratch_mutex;
+void* g_scratch_ptr[kMaxDevices] = {};
 
 }  // namespace
 
@@ -50,16 +50,24 @@ extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v,
     // image on the device if it is not loaded yet).
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
-    ScratchAddress& slot = g_scratch[dev];
-    std::call_once(slot.once, [&] {
-        slot.err = cudaGetSymbolAddress(&slot.ptr, g_noalloc_scratch);
-    });
-    if (slot.err != cudaSuccess || slot.ptr == nullptr) return FA_ERR_CUDA;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_scratch_mutex);
+        if (g_scratch_ptr[dev] == nullptr) {
+            void* ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+                (void)cudaGetLastError();  // do not leave the lookup's error behind
+                return FA_ERR_CUDA;
+            }
+            g_scratch_ptr[dev] = ptr;
+        }
+        scratch = g_scratch_ptr[dev];
+    }
 
     // The existing backward pass, pointed at the scratch array.  Its first
     // stage rewrites every workspace word it later reads (it zeroes the dQ
     // accumulator and refills the row vectors), so leftovers from an earlier
     // call never leak into this one.
-    return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, slot.ptr,
+    return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, B, H, N, d, causal, scale, scratch,
                   kScratchBytes, stream);
 }

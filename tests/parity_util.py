@@ -5,11 +5,23 @@ Tolerances (GPU result vs the fp64 oracle on the same seeded inputs):
   O:            max-abs <= 1e-2 and relative L2 <= 5e-3
   dQ, dK, dV:   max-abs <= 2e-2
   LSE:          max-abs <= 1e-3 (fp32 statistic; the kernel's error is ~1e-5)
-Outputs are bf16, whose own rounding of an exact value is up to half an ulp:
-0.0156 for |x| in [4, 8) and 0.031 above 8, at or above the 2e-2 bound.  The
-max-abs bounds therefore apply to each element's error in excess of that
-element's unavoidable rounding, |gpu - ref| - |bf16(ref) - ref| (the "excess");
-the raw max-abs and the bf16 floor max|bf16(ref) - ref| are reported beside it.
+
+The max-abs bounds are asserted on the raw error |gpu - ref| of every element
+small enough for the bf16 output format to leave room for the arithmetic:
+|ref| < 4 for O and |ref| < 2 for the gradients.  The error of a bf16 output
+is its arithmetic error plus up to half an ulp of rounding; half an ulp is
+2^-8 = 0.0039 for |x| in [1, 2), 2^-7 = 0.0078 in [2, 4) and 2^-6 = 0.0156
+in [4, 8).  O's arithmetic stays within ~2e-3, so |ref| < 4 leaves it room.  The gradients'
+arithmetic -- fp32 sums of products whose P and dS operands are rounded to
+bf16, 2^-8 relative each, over up to N terms -- reaches ~0.016 at d = 64
+with the causal mask (where dP = dO.v has standard deviation 8), so only
+|ref| < 2 (half an ulp at most 2^-8 = 0.0039) leaves the bound for it.
+From those magnitudes on the bound applies to the error in excess of that
+element's own rounding, |gpu - ref| - |bf16(ref) - ref|.  Relative L2 is
+always raw.  Every check records its figures -- raw max-abs over all
+elements, over the raw-bound region and per magnitude band ([0,1), [1,2),
+[2,4), [4,8), [8,inf)), the excess above the region, the bf16 floor,
+relative L2 -- in ``parity_log``.
 """
 from __future__ import annotations
 
@@ -19,16 +31,26 @@ import torch
 import oracle
 import exact_attention_109_b200 as fa
 from exact_attention_109_b200.inputs import attention_inputs, default_scale, to_f64
+import parity_log
 
 TOL_O_MAX = 1e-2
 TOL_O_REL_L2 = 5e-3
 TOL_GRAD_MAX = 2e-2
 TOL_LSE_MAX = 1e-3
+# Magnitude below which the max-abs bound holds for the raw error.
+RAW_BELOW_O = 4.0
+RAW_BELOW_GRAD = 2.0
+BANDS = (0.0, 1.0, 2.0, 4.0, 8.0, float("inf"))
+
+
+def bf16_round(ref: np.ndarray) -> np.ndarray:
+    r = torch.from_numpy(np.ascontiguousarray(ref, dtype=np.float64))
+    return r.to(torch.bfloat16).to(torch.float64).numpy()
 
 
 def bf16_floor(ref: np.ndarray) -> float:
-    r = torch.from_numpy(np.ascontiguousarray(ref)).to(torch.bfloat16).to(torch.float64)
-    return float(np.max(np.abs(r.numpy() - ref))) if ref.size else 0.0
+    ref = np.asarray(ref, dtype=np.float64)
+    return float(np.max(np.abs(bf16_round(ref) - ref))) if ref.size else 0.0
 
 
 def max_abs(a, b) -> float:
@@ -42,19 +64,97 @@ def max_abs(a, b) -> float:
 
 def max_excess(gpu, ref) -> float:
     """max over elements of |gpu - ref| - |bf16(ref) - ref|."""
-    gpu = np.asarray(gpu, dtype=np.float64)
-    ref = np.ascontiguousarray(ref, dtype=np.float64)
-    if gpu.size == 0:
-        return 0.0
-    assert np.all(np.isfinite(gpu)), "non-finite values in GPU output"
-    rounded = torch.from_numpy(ref).to(torch.bfloat16).to(torch.float64).numpy()
-    return float(np.max(np.abs(gpu - ref) - np.abs(rounded - ref)))
+    figs = error_figures(gpu, ref, raw_below=0.0)
+    return figs["excess_above"]
 
 
 def rel_l2(a, b) -> float:
     a = np.asarray(a, dtype=np.float64)
     b = np.asarray(b, dtype=np.float64)
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def error_figures(gpu, ref, raw_below: float) -> dict:
+    """Raw max-abs over all elements ("max") and over |ref| < raw_below
+    ("max_below"); max of |gpu-ref| - |bf16(ref)-ref| over |ref| >= raw_below
+    ("excess_above", 0 when there is no such element); the bf16 floor
+    max|bf16(ref) - ref| ("floor"); relative L2 ("rel_l2")."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    if gpu.size == 0:
+        return {"max": 0.0, "max_below": 0.0, "excess_above": 0.0, "floor": 0.0,
+                "rel_l2": 0.0, "n_above": 0}
+    assert np.all(np.isfinite(gpu)), "non-finite values in GPU output"
+    err = np.abs(gpu - ref)
+    floor = np.abs(bf16_round(ref) - ref)
+    mag = np.abs(ref)
+    below = mag < raw_below
+    above = ~below
+    figs = {
+        "max": float(err.max()),
+        "max_below": float(err[below].max()) if below.any() else 0.0,
+        "excess_above": float((err - floor)[above].max()) if above.any() else 0.0,
+        "floor": float(floor.max()),
+        "rel_l2": rel_l2(gpu, ref),
+        "n_above": int(above.sum()),
+    }
+    for lo, hi in zip(BANDS[:-1], BANDS[1:]):
+        band = (mag >= lo) & (mag < hi)
+        if band.any():
+            figs[f"max_mag{lo:g}to{hi:g}"] = float(err[band].max())
+    return figs
+
+
+class Check:
+    """Accumulates the figures of one parity check and the bounds they
+    break; ``done()`` records them and fails the test on any breach."""
+
+    def __init__(self):
+        self.res: dict = {}
+        self.fails: list = []
+
+    def _merge(self, name, figs):
+        for key, val in figs.items():
+            k = f"{name}_{key}"
+            self.res[k] = max(self.res.get(k, val), val)
+
+    def output(self, name, gpu, ref, tol, raw_below, rel_tol=None):
+        figs = error_figures(gpu, ref, raw_below)
+        self._merge(name, figs)
+        if figs["max_below"] > tol:
+            self.fails.append(f"{name}: raw max-abs {figs['max_below']:.3g} > {tol} "
+                              f"over |ref| < {raw_below}")
+        if figs["excess_above"] > tol:
+            self.fails.append(f"{name}: error beyond the bf16 floor "
+                              f"{figs['excess_above']:.3g} > {tol} over |ref| >= {raw_below}")
+        if rel_tol is not None and figs["rel_l2"] > rel_tol:
+            self.fails.append(f"{name}: rel-L2 {figs['rel_l2']:.3g} > {rel_tol}")
+        return figs
+
+    def o(self, gpu, ref, name="o"):
+        return self.output(name, gpu, ref, TOL_O_MAX, RAW_BELOW_O, TOL_O_REL_L2)
+
+    def grad(self, name, gpu, ref):
+        return self.output(name, gpu, ref, TOL_GRAD_MAX, RAW_BELOW_GRAD)
+
+    def lse(self, gpu, ref, name="lse"):
+        err = max_abs(gpu, ref)
+        k = f"{name}_max"
+        self.res[k] = max(self.res.get(k, err), err)
+        if err > TOL_LSE_MAX:
+            self.fails.append(f"{name}: max-abs {err:.3g} > {TOL_LSE_MAX}")
+        return err
+
+    def bound(self, name, value, limit):
+        self.res[name] = max(self.res.get(name, value), value)
+        if not value <= limit:
+            self.fails.append(f"{name}: {value:.3g} > {limit}")
+
+    def done(self):
+        parity_log.record(self.res)
+        assert not self.fails, (self.fails, self.res)
+        return self.res
 
 
 def gpu_inputs(B, H, N, d, seed, dist="normal", with_dout=False):
@@ -87,18 +187,28 @@ def run_backward(dev, out, lse, causal, scale):
 
 
 def check_forward_full(host, o, lse, causal, scale):
-    """Whole-tensor comparison; returns a dict of error figures."""
+    """Whole-tensor comparison of O and LSE; returns the error figures."""
     o_ref, lse_ref = oracle.ref_fwd(to_f64(host["q"]), to_f64(host["k"]),
                                     to_f64(host["v"]), causal, scale)
-    o_gpu = to_f64(o.cpu())
-    lse_gpu = lse.cpu().double().numpy()
-    res = {"o_excess": max_excess(o_gpu, o_ref), "o_max": max_abs(o_gpu, o_ref),
-           "o_rel_l2": rel_l2(o_gpu, o_ref), "lse_max": max_abs(lse_gpu, lse_ref),
-           "o_floor": bf16_floor(o_ref)}
-    assert res["o_excess"] <= TOL_O_MAX, res
-    assert res["o_rel_l2"] <= TOL_O_REL_L2, res
-    assert res["lse_max"] <= TOL_LSE_MAX, res
-    return res
+    c = Check()
+    c.o(to_f64(o.cpu()), o_ref)
+    c.lse(lse.cpu().double().numpy(), lse_ref)
+    return c.done()
+
+
+def check_full(host, o, lse, dq, dk, dv, causal, scale):
+    """Whole-tensor comparison of O, LSE, dQ, dK and dV (every element of
+    every head) against one oracle forward and backward."""
+    args = [to_f64(host[x]) for x in ("q", "k", "v")]
+    o_ref, lse_ref = oracle.ref_fwd(*args, causal, scale)
+    c = Check()
+    c.o(to_f64(o.cpu()), o_ref)
+    c.lse(lse.cpu().double().numpy(), lse_ref)
+    del o_ref, lse_ref
+    refs = oracle.ref_bwd(*args, to_f64(host["dO"]), causal, scale)[:3]
+    for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs):
+        c.grad(name, to_f64(got.cpu()), ref)
+    return c.done()
 
 
 def sample_rows(N, count, rng):
@@ -115,40 +225,28 @@ def check_forward_sampled(host, o, lse, causal, scale, heads, rows_per_head, see
     q, k, v = (host[x].reshape(B * H, N, d) for x in "qkv")
     o_gpu = o.reshape(B * H, N, d)
     lse_gpu = lse.reshape(B * H, N)
-    worst = {"o_excess": 0.0, "o_max": 0.0, "lse_max": 0.0, "o_rel_l2": 0.0}
+    c = Check()
     for bh in heads:
         rows = sample_rows(N, rows_per_head, rng)
         o_ref, l_ref = oracle.ref_fwd_rows(to_f64(q[bh]), to_f64(k[bh]),
                                            to_f64(v[bh]), rows, causal, scale)
-        og = to_f64(o_gpu[bh][torch.from_numpy(rows).to(o.device)].cpu())
-        lg = lse_gpu[bh][torch.from_numpy(rows).to(o.device)].cpu().double().numpy()
-        worst["o_excess"] = max(worst["o_excess"], max_excess(og, o_ref))
-        worst["o_max"] = max(worst["o_max"], max_abs(og, o_ref))
-        worst["o_rel_l2"] = max(worst["o_rel_l2"], rel_l2(og, o_ref))
-        worst["lse_max"] = max(worst["lse_max"], max_abs(lg, l_ref))
-    assert worst["o_excess"] <= TOL_O_MAX, worst
-    assert worst["o_rel_l2"] <= TOL_O_REL_L2, worst
-    assert worst["lse_max"] <= TOL_LSE_MAX, worst
-    return worst
+        idx = torch.from_numpy(rows).to(o.device)
+        c.o(to_f64(o_gpu[bh][idx].cpu()), o_ref)
+        c.lse(lse_gpu[bh][idx].cpu().double().numpy(), l_ref)
+    return c.done()
 
 
 def check_backward_heads(host, dq, dk, dv, causal, scale, heads):
     """Whole-head gradient comparison for the listed (flattened) heads."""
     B, H, N, d = host["q"].shape
     flat = {x: host[x].reshape(B * H, 1, N, d) for x in ("q", "k", "v", "dO")}
-    res = {f"{n}_{m}": 0.0 for n in ("dq", "dk", "dv") for m in ("excess", "max")}
-    res["floor"] = 0.0
+    c = Check()
     for bh in heads:
         args = [to_f64(flat[x][bh:bh + 1]) for x in ("q", "k", "v", "dO")]
         rq, rk, rv, _ = oracle.ref_bwd(*args, causal, scale)
         for name, got, ref in (("dq", dq, rq), ("dk", dk, rk), ("dv", dv, rv)):
-            g = to_f64(got.reshape(B * H, 1, N, d)[bh:bh + 1].cpu())
-            res[name + "_excess"] = max(res[name + "_excess"], max_excess(g, ref))
-            res[name + "_max"] = max(res[name + "_max"], max_abs(g, ref))
-            res["floor"] = max(res["floor"], bf16_floor(ref))
-    for name in ("dq", "dk", "dv"):
-        assert res[name + "_excess"] <= TOL_GRAD_MAX, res
-    return res
+            c.grad(name, to_f64(got.reshape(B * H, 1, N, d)[bh:bh + 1].cpu()), ref)
+    return c.done()
 
 
 def check_backward_sampled(host, dq, dk, dv, causal, scale, heads, rows_per_head, seed=0):
@@ -156,7 +254,7 @@ def check_backward_sampled(host, dq, dk, dv, causal, scale, heads, rows_per_head
     B, H, N, d = host["q"].shape
     rng = np.random.default_rng(seed)
     flat = {x: host[x].reshape(B * H, N, d) for x in ("q", "k", "v", "dO")}
-    res = {f"{n}_{m}": 0.0 for n in ("dq", "dk", "dv") for m in ("excess", "max")}
+    c = Check()
     for bh in heads:
         q, k, v, dO = (to_f64(flat[x][bh]) for x in ("q", "k", "v", "dO"))
         rows = sample_rows(N, rows_per_head, rng)
@@ -165,12 +263,8 @@ def check_backward_sampled(host, dq, dk, dv, causal, scale, heads, rows_per_head
         rdq = oracle.ref_dq_rows(q, k, v, dO, rows, causal, scale)
         rdk, rdv = oracle.ref_dkdv_rows(q, k, v, dO, lse_h, D_h, rows, causal, scale)
         for name, got, ref in (("dq", dq, rdq), ("dk", dk, rdk), ("dv", dv, rdv)):
-            g = to_f64(got.reshape(B * H, N, d)[bh].cpu()[idx])
-            res[name + "_excess"] = max(res[name + "_excess"], max_excess(g, ref))
-            res[name + "_max"] = max(res[name + "_max"], max_abs(g, ref))
-    for name in ("dq", "dk", "dv"):
-        assert res[name + "_excess"] <= TOL_GRAD_MAX, res
-    return res
+            c.grad(name, to_f64(got.reshape(B * H, N, d)[bh].cpu()[idx]), ref)
+    return c.done()
 
 
 def check_backward_causal_tail(host, dq, dk, dv, scale, heads, rows_per_head, tail, seed=0):
@@ -182,7 +276,7 @@ def check_backward_causal_tail(host, dq, dk, dv, scale, heads, rows_per_head, ta
     first = N - tail
     rng = np.random.default_rng(seed)
     flat = {x: host[x].reshape(B * H, N, d) for x in ("q", "k", "v", "dO")}
-    res = {f"{n}_{m}": 0.0 for n in ("dq", "dk", "dv") for m in ("excess", "max")}
+    c = Check()
     for bh in heads:
         q, k, v, dO = (to_f64(flat[x][bh]) for x in ("q", "k", "v", "dO"))
         q_rows = sample_rows(N, rows_per_head, rng)
@@ -192,9 +286,6 @@ def check_backward_causal_tail(host, dq, dk, dv, scale, heads, rows_per_head, ta
         rdk, rdv = oracle.ref_dkdv_rows(q, k, v, dO, lse_h, D_h, k_rows, True, scale)
         for name, got, ref, rows in (("dq", dq, rdq, q_rows), ("dk", dk, rdk, k_rows),
                                      ("dv", dv, rdv, k_rows)):
-            g = to_f64(got.reshape(B * H, N, d)[bh].cpu()[torch.from_numpy(rows)])
-            res[name + "_excess"] = max(res[name + "_excess"], max_excess(g, ref))
-            res[name + "_max"] = max(res[name + "_max"], max_abs(g, ref))
-    for name in ("dq", "dk", "dv"):
-        assert res[name + "_excess"] <= TOL_GRAD_MAX, res
-    return res
+            c.grad(name, to_f64(got.reshape(B * H, N, d)[bh].cpu()[torch.from_numpy(rows)]),
+                   ref)
+    return c.done()

@@ -3,7 +3,8 @@ against the oracle's ref_fwd_bias / ref_bwd_bias (pinned to brute force,
 torch autograd and finite differences) on the same seeded bf16 inputs, for
 full and broadcast biases, both masks, d = 64 and 128, ragged lengths, and
 biases that hide keys with -inf.  Tolerances are those of the plain path;
-dBias is a gradient (dS) and takes the gradient bound."""
+dBias is a gradient (dS) and takes the gradient bound.  No oracle call is
+given anything the CUDA path computed."""
 import numpy as np
 import pytest
 import torch
@@ -11,8 +12,7 @@ import torch
 import oracle
 import exact_attention_109_b200 as fa
 from exact_attention_109_b200.inputs import attention_inputs, default_scale, to_f64
-from parity_util import (TOL_GRAD_MAX, TOL_LSE_MAX, TOL_O_MAX, TOL_O_REL_L2, max_abs, max_excess,
-                         rel_l2)
+from parity_util import Check
 
 pytestmark = pytest.mark.gpu
 
@@ -38,29 +38,36 @@ def _run(B, H, N, d, causal, bshape, seed, hide=0.0, backward=True):
     assert fa.fa_get_device_error() == fa.FA_OK
     args = [to_f64(host[x]) for x in ("q", "k", "v")]
     o_ref, lse_ref = oracle.ref_fwd_bias(*args, to_f64(bias), causal, scale)
-    og = to_f64(o.cpu())
-    res = {"o_excess": max_excess(og, o_ref), "o_rel_l2": rel_l2(og, o_ref),
-           "lse": max_abs(lse.cpu().double().numpy(), lse_ref)}
-    assert res["o_excess"] <= TOL_O_MAX, res
-    assert res["o_rel_l2"] <= TOL_O_REL_L2, res
-    assert res["lse"] <= TOL_LSE_MAX, res
+    c = Check()
+    c.o(to_f64(o.cpu()), o_ref)
+    c.lse(lse.cpu().double().numpy(), lse_ref)
     if not backward:
-        return res
+        return c.done()
     dq, dk, dv, db = fa.attention_backward_bias(q, k, v, bd, o, lse, dO, causal, scale)
     assert fa.fa_get_device_error() == fa.FA_OK
     refs = oracle.ref_bwd_bias(*args, to_f64(bias), to_f64(host["dO"]), causal, scale)
     for name, got, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), refs[:3]):
-        res[name] = max_excess(to_f64(got.cpu()), ref)
-        assert res[name] <= TOL_GRAD_MAX, (name, res)
-    # dBias is dS itself, not damped by the 1/sqrt(d) of dQ and dK: the
-    # reference takes D = rowsum(dO * O) from the bf16 O the backward pass
-    # receives, as the kernel must (the exact-O value moves dS by up to
-    # P_ij * 2^-9 * sum |dO| |O| in a row whose softmax is peaked).
-    ref_db = oracle.ref_bwd_bias(*args, to_f64(bias), to_f64(host["dO"]), causal, scale,
-                                 o_given=to_f64(o.cpu()))[3]
-    res["dbias"] = max_excess(to_f64(db.cpu()), ref_db)
-    assert res["dbias"] <= TOL_GRAD_MAX, res
-    return res
+        c.grad(name, to_f64(got.cpu()), ref)
+    # dBias is dS itself, not damped by the 1/sqrt(d) of dQ and dK, and
+    # D = rowsum(dO * O) enters it undamped: one bf16 ulp of one element of
+    # the O a backward pass receives moves dS_ij by P_ij |dO| ulp, up to
+    # ~0.03 in rows whose softmax is peaked.  So dBias is checked on a second
+    # backward pass whose O and LSE inputs are the oracle's own forward
+    # results in the formats the pass takes (O rounded to bf16, LSE to fp32),
+    # against the oracle's dBias with D taken from that same bf16 O.  Both
+    # sides then start from identical inputs; nothing computed by the CUDA
+    # path enters the oracle.
+    o_in = torch.from_numpy(o_ref).to(torch.bfloat16)
+    lse_in = torch.from_numpy(lse_ref).to(torch.float32)
+    dq2, dk2, dv2, db = fa.attention_backward_bias(q, k, v, bd, o_in.cuda(), lse_in.cuda(), dO,
+                                                   causal, scale)
+    assert fa.fa_get_device_error() == fa.FA_OK
+    refs2 = oracle.ref_bwd_bias(*args, to_f64(bias), to_f64(host["dO"]), causal, scale,
+                                o_given=to_f64(o_in))
+    for name, got, ref in zip(("dq_oracle_o", "dk_oracle_o", "dv_oracle_o", "dbias"),
+                              (dq2, dk2, dv2, db), refs2):
+        c.grad(name, to_f64(got.cpu()), ref)
+    return c.done()
 
 
 @pytest.mark.parametrize("d", [64, 128])

@@ -14,8 +14,7 @@ import torch
 import oracle
 import exact_attention_109_b200 as fa
 from exact_attention_109_b200.inputs import decode_inputs, default_scale, to_f64
-from parity_util import (TOL_LSE_MAX, TOL_O_MAX, TOL_O_REL_L2, max_abs, max_excess,
-                         rel_l2)
+from parity_util import Check, max_abs
 
 pytestmark = pytest.mark.gpu
 
@@ -42,14 +41,10 @@ def run_decode(host, causal, scale, kv_rows=None, n_keys=None, dist_fill=float("
 def check_decode(host, o, lse, causal, scale):
     o_ref, lse_ref = oracle.ref_fwd_decode(to_f64(host["q"]), to_f64(host["k"]),
                                            to_f64(host["v"]), causal, scale)
-    o_gpu = to_f64(o.cpu())
-    lse_gpu = lse.cpu().double().numpy()
-    res = {"o_excess": max_excess(o_gpu, o_ref), "o_max": max_abs(o_gpu, o_ref),
-           "o_rel_l2": rel_l2(o_gpu, o_ref), "lse_max": max_abs(lse_gpu, lse_ref)}
-    assert res["o_excess"] <= TOL_O_MAX, res
-    assert res["o_rel_l2"] <= TOL_O_REL_L2, res
-    assert res["lse_max"] <= TOL_LSE_MAX, res
-    return res
+    c = Check()
+    c.o(to_f64(o.cpu()), o_ref)
+    c.lse(lse.cpu().double().numpy(), lse_ref)
+    return c.done()
 
 
 @pytest.mark.parametrize("d", [64, 128])

@@ -711,3 +711,28 @@ def test_bias_gradient_by_finite_differences():
     o, _ = oracle.ref_fwd_bias(q, k, v, bias, True, 0.8)
     db2 = oracle.ref_bwd_bias(q, k, v, bias, dO, True, 0.8, o_given=o)[3]
     assert rel_err(db2, db) <= 1e-14
+
+
+def test_dbias_with_bf16_rounded_o_stays_within_the_rounding_bound():
+    """The dBias reference of the GPU tests takes D = rowsum(dO * O) from the
+    oracle's own O rounded to bf16 (the format the backward receives O in).
+    bf16 keeps 8 significant bits, so |bf16(x) - x| <= 2^-8 |x| and
+    dS_ij moves by at most P_ij * 2^-8 * sum_d |dO_id| |O_id|.  This pins
+    that reference to the exact-D one within that bound, and shows that the
+    rounding really reaches it (the model is not the exact D in disguise)."""
+    q, k, v, dO = rng_inputs(705, 2, 3, 24, 16)
+    bias = np.random.default_rng(5).standard_normal((2, 3, 24, 24)) * 2
+    for causal in (False, True):
+        o, lse = oracle.ref_fwd_bias(q, k, v, bias, causal, 0.6)
+        o_bf16 = torch.from_numpy(o).to(torch.bfloat16).to(torch.float64).numpy()
+        assert np.all(np.abs(o_bf16 - o) <= 2.0 ** -8 * np.abs(o))
+        db_exact = oracle.ref_bwd_bias(q, k, v, bias, dO, causal, 0.6)[3]
+        db_model = oracle.ref_bwd_bias(q, k, v, bias, dO, causal, 0.6, o_given=o_bf16)[3]
+        s = 0.6 * np.einsum("bhid,bhjd->bhij", q, k) + bias
+        if causal:
+            s = np.where(np.arange(24)[None, :] > np.arange(24)[:, None], -np.inf, s)
+        p = np.exp(s - lse[..., None])
+        bound = p * 2.0 ** -8 * np.sum(np.abs(dO) * np.abs(o), axis=-1, keepdims=True)
+        diff = np.abs(db_model - db_exact)
+        assert np.all(diff <= bound * (1 + 1e-9) + 1e-15)
+        assert diff.max() > 0.05 * bound.max()
