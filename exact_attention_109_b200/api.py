@@ -262,9 +262,11 @@ def _require(ts, shape, dtype, device):
             raise ValueError(f"{name}: expected shape {shape}, got {tuple(t.shape)}")
 
 
-def attention_forward(q, k, v, causal: bool, scale: float, out=None, lse=None,
+def attention_forward(q, k, v, causal: int, scale: float, out=None, lse=None,
                       stream=None):
-    """O, LSE = fa_fwd(q, k, v) for CUDA bf16 [B,H,N,d] tensors."""
+    """O, LSE = fa_fwd(q, k, v) for CUDA bf16 [B,H,N,d] tensors.  causal:
+    0 / False none, 1 / True key j visible to query i iff j <= i, 2 iff
+    j < i (row 0 then sees no key: O = 0, LSE = -inf)."""
     B, H, N, d = _shape(q)
     _require({"q": q, "k": k, "v": v}, (B, H, N, d), torch.bfloat16, q.device)
     if out is None:
@@ -279,9 +281,10 @@ def attention_forward(q, k, v, causal: bool, scale: float, out=None, lse=None,
     return out, lse
 
 
-def attention_backward(q, k, v, out, lse, dO, causal: bool, scale: float,
+def attention_backward(q, k, v, out, lse, dO, causal: int, scale: float,
                        dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """dQ, dK, dV = fa_bwd(...) for CUDA bf16 [B,H,N,d] tensors."""
+    """dQ, dK, dV = fa_bwd(...) for CUDA bf16 [B,H,N,d] tensors (causal as
+    for attention_forward)."""
     B, H, N, d = _shape(q)
     _require({"q": q, "k": k, "v": v, "out": out, "dO": dO}, (B, H, N, d),
              torch.bfloat16, q.device)

@@ -236,6 +236,7 @@ fa::FwdParams fwd_params(float* lse, unsigned int* err, int N, long long bh, int
     prm.H = H;
     prm.bias_batch = 0;
     prm.bias_heads = 0;
+    prm.strict = 0;
     return prm;
 }
 
@@ -262,7 +263,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     if (st != FA_OK) return st;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return FA_ERR_MISALIGNED;
-    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (causal < 0 || causal > 2) return FA_ERR_INVALID_ARG;
     int dev;
     unsigned int* err;
     if ((st = device_setup(&dev, &err)) != FA_OK) return st;
@@ -273,7 +274,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     if (!encode_bf16(&mq, q, d, N, bh, 128) || !encode_bf16(&mk, k, d, N, bh, 128) ||
         !encode_bf16(&mv, v, d, N, bh, 128) || !encode_bf16(&mo, o, d, N, bh, 32))
         return FA_ERR_CUDA;
-    const fa::FwdParams prm = fwd_params(lse, err, N, bh, H, scale * 1.4426950408889634f);
+    fa::FwdParams prm = fwd_params(lse, err, N, bh, H, scale * 1.4426950408889634f);
+    prm.strict = causal == 2;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     if (d == 64)
@@ -401,7 +403,7 @@ fa_status bwd_main_impl(const void* q, const void* k, const void* v, const void*
                         const void* bias = nullptr, void* dbias = nullptr, int bias_batch = 0,
                         int bias_heads = 0) {
     if (!q || !k || !v || !dO || !dk || !dv) return FA_ERR_INVALID_ARG;
-    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (causal < 0 || causal > (bias ? 1 : 2)) return FA_ERR_INVALID_ARG;
     fa::BwdWorkspace ws;
     int dev;
     unsigned int* err;
@@ -425,7 +427,7 @@ fa_status bwd_main_impl(const void* q, const void* k, const void* v, const void*
     cudaError_t e;
 #define FA_BWD_MAIN(DD, CC, BB)                                                            \
     fa::launch_bwd_main<DD, CC, BB>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv, macc, err, s, \
-                                    0, bias, dbias, H, bias_batch, bias_heads)
+                                    0, bias, dbias, H, bias_batch, bias_heads, causal == 2)
     if (bias) {
         if (d == 64)
             e = causal ? FA_BWD_MAIN(64, true, true) : FA_BWD_MAIN(64, false, true);
@@ -462,7 +464,8 @@ fa_status bwd_accum_impl(const void* q, const void* k, const void* v, const void
                          float* dk_acc, float* dv_acc, int B, int H, int N, int d, int causal,
                          float scale, void* workspace, size_t workspace_bytes, void* stream) {
     if (!q || !k || !v || !dO || !dk_acc || !dv_acc) return FA_ERR_INVALID_ARG;
-    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (causal < 0 || causal > 2) return FA_ERR_INVALID_ARG;
+    const int strict = causal == 2;
     fa::BwdWorkspace ws;
     int dev;
     unsigned int* err;
@@ -485,16 +488,14 @@ fa_status bwd_accum_impl(const void* q, const void* k, const void* v, const void
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const int ibh = static_cast<int>(bh);
     cudaError_t e;
+#define FA_BWD_ACC(DD, CC)                                                                  \
+    fa::launch_bwd_main<DD, CC>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv, macc, err, s, 1, \
+                                nullptr, nullptr, 1, 0, 0, strict)
     if (d == 64)
-        e = causal ? fa::launch_bwd_main<64, true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
-                                                   macc, err, s, 1)
-                   : fa::launch_bwd_main<64, false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
-                                                    macc, err, s, 1);
+        e = causal ? FA_BWD_ACC(64, true) : FA_BWD_ACC(64, false);
     else
-        e = causal ? fa::launch_bwd_main<128, true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
-                                                    macc, err, s, 1)
-                   : fa::launch_bwd_main<128, false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk,
-                                                     mdv, macc, err, s, 1);
+        e = causal ? FA_BWD_ACC(128, true) : FA_BWD_ACC(128, false);
+#undef FA_BWD_ACC
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -575,7 +576,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
         return FA_ERR_INVALID_ARG;
     fa_status st = check_sizes(B, H, N, d, scale);
     if (st != FA_OK) return st;
-    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    if (causal < 0 || causal > 2) return FA_ERR_INVALID_ARG;
     if (workspace_bytes < fa::bwd_workspace_bytes(static_cast<long long>(B) * H, N, d))
         return FA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) ||

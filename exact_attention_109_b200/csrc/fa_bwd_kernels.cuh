@@ -209,6 +209,7 @@ struct BwdParams {
     int bias_heads;
     float scale;
     float scale_log2;
+    int strict;      // causal mask without the diagonal: key j visible iff j < i
 };
 
 // BIAS: an additive score bias (and optionally its gradient), see BwdParams.
@@ -507,7 +508,8 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
                                                                32 * g);
             const float4* d4 = l4 + T::BM / 4;
             const int qrow0 = (qb0 + k) * T::BM + 32 * g;
-            const int masked = CAUSAL ? kv_row - qrow0 : 0;  // columns e < masked are hidden
+            // columns e < masked are hidden (strict: the diagonal too)
+            const int masked = CAUSAL ? kv_row - qrow0 + p.strict : 0;
             uint32_t pk[16], dk[16];
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
@@ -707,7 +709,7 @@ cudaError_t launch_bwd_main(int bh, int N, float scale, const BwdWorkspace& ws,
                             const CUtensorMap& mdv, const CUtensorMap& macc, unsigned int* err,
                             cudaStream_t s, int accum = 0, const void* bias = nullptr,
                             void* dbias = nullptr, int H = 1, int bias_batch = 0,
-                            int bias_heads = 0) {
+                            int bias_heads = 0, int strict = 0) {
     using T = BwdTraits<D>;
     BwdParams prm;
     prm.lse2 = ws.lse2;
@@ -726,6 +728,7 @@ cudaError_t launch_bwd_main(int bh, int N, float scale, const BwdWorkspace& ws,
     prm.bias_heads = bias_heads;
     prm.scale = scale;
     prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.strict = strict;
     const long long grid = static_cast<long long>(bh) * prm.n_kv;
     fa_bwd_main_kernel<D, CAUSAL, BIAS><<<static_cast<unsigned>(grid), T::NUM_THREADS,
                                           T::SMEM_BYTES, s>>>(

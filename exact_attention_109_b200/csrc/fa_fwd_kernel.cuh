@@ -98,6 +98,7 @@ struct FwdParams {
     int H;                 // heads (to split b*H + h)
     int bias_batch;        // bias varies with the batch index (else shared)
     int bias_heads;        // bias varies with the head index (else shared)
+    int strict;            // causal mask without the diagonal: key j visible iff j < i
 };
 
 // One softmax row over a 128-key block: p = exp2(s * scale*log2(e) - m) in
@@ -501,7 +502,7 @@ __global__ void __launch_bounds__(384, 1)
                 (kv0 + T::BN > N) || (CAUSAL && kv0 + T::BN - 1 > row0);
             if (masked_block) {
                 int lim = min(T::BN, N - kv0);
-                if (CAUSAL) lim = min(lim, row - kv0 + 1);
+                if (CAUSAL) lim = min(lim, row - kv0 + 1 - p.strict);
 #pragma unroll
                 for (int c = 0; c < 128; ++c)
                     if (c >= lim) sr[c >> 5][c & 31] = __float_as_uint(-INFINITY);
@@ -538,7 +539,10 @@ __global__ void __launch_bounds__(384, 1)
                 }
             }
             m = m_new;
-            softmax_block_exp<T::PSPLIT>(sr, sl2e, m, s_tm, l, lr, &p_half[t]);
+            // A row that has seen no visible key yet (only the strict causal
+            // mask's row 0) keeps m = -inf; its weights are exp2(-inf) = 0.
+            softmax_block_exp<T::PSPLIT>(sr, sl2e, m == -INFINITY ? 0.f : m, s_tm, l, lr,
+                                         &p_half[t]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_ready[t]);
@@ -547,7 +551,10 @@ __global__ void __launch_bounds__(384, 1)
         if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&o_final[t], 0, st));
         if (ok) {
             tc_fence_after();
-            const float inv_l = 1.0f / lr;
+            // A row with no visible key (strict causal row 0) keeps m = -inf:
+            // O = 0, LSE = -inf.  (Its weights are not all 0 -- the FMA-pipe
+            // exp2 returns 2^-126 for -inf -- so lr alone cannot tell.)
+            const float inv_l = m == -INFINITY ? 0.f : 1.0f / lr;
             const float lse_val = (m + log2f(l)) * 0.6931471805599453f;
             // Stage O (bf16, 128-byte swizzle) in this tile's Q buffer, which
             // no MMA reads any more (e4m3 scores: in the staging region),

@@ -9,10 +9,21 @@ is an ordinary attention problem of the shard length, computed by the CUDA
 library (``fa_fwd`` / ``fa_bwd_main_accumulate``); the pairs' results are
 folded together with the log-sum-exp rule (``fa_lse_merge``).
 
-Layout: rank r of a ring of G holds positions [r n, (r+1) n) of a sequence of
-G n tokens: q, k, v, dO, O as [B, H, n, d] bf16, LSE as [B, H, n] fp32.
-Causal masking is by global position, so for query shard r the key shards
-j < r are fully visible, shard r is causal, and shards j > r are skipped.
+Layouts of the sequence over a ring of G ranks (every rank holds n = N / G
+positions as q, k, v, dO, O [B, H, n, d] bf16 and LSE [B, H, n] fp32):
+
+* "contiguous": rank r holds positions [r n, (r+1) n).  Under the causal mask
+  key shard j is fully visible to query shard r when j < r, causal when
+  j = r and skipped when j > r, so rank r computes r + 1 pairs and the last
+  rank's G pairs are the ring's critical path.
+* "striped": rank r holds positions r, r + G, r + 2G, ... (local row i is
+  position i G + r).  Key j of shard s is then visible to query i of shard r
+  iff j G + s <= i G + r: j <= i when s <= r, j < i when s > r.  Every pair is
+  half a block of work -- causal with or without its diagonal -- so every
+  rank computes the same G half blocks and the causal ring is balanced (the
+  striped layout of "Striped Attention: Faster Ring Attention for Causal
+  Transformers", Brandon et al., 2023; not on the pages, which give only the
+  Ring Attention abstract).
 
 Each rank's schedule is written once, as a generator (``forward_program`` /
 ``backward_program``) that yields at its exchange points:
@@ -95,17 +106,36 @@ class CudaOps:
 # ---------------------------------------------------------------- schedules
 
 
-def _visible(causal: bool, rank: int, shard: int) -> bool:
-    return (not causal) or shard <= rank
+LAYOUTS = ("contiguous", "striped")
 
 
-def _last_visible_step(causal: bool, rank: int, world: int) -> int:
-    # step s holds key shard (rank - s) mod world; causal ranks see s = 0..rank
-    return rank if causal else world - 1
+def pair_mask(causal: bool, layout: str, rank: int, shard: int):
+    """Mask of the pair (query shard `rank`, key shard `shard`) as the
+    library's `causal` argument -- 0 none, 1 causal (j <= i), 2 causal
+    without the diagonal (j < i) -- or None when no key of the shard is
+    visible (the pair is skipped)."""
+    if layout not in LAYOUTS:
+        raise ValueError(f"unknown ring layout {layout!r}")
+    if not causal:
+        return 0
+    if layout == "striped":
+        return 1 if shard <= rank else 2
+    if shard < rank:
+        return 0
+    return 1 if shard == rank else None
 
 
-def forward_program(q, k, v, causal: bool, scale: float, rank: int, world: int, ops=None):
-    """Rank `rank`'s forward: returns (O bf16, LSE fp32) of its query shard."""
+def _last_visible_step(causal: bool, layout: str, rank: int, world: int) -> int:
+    # step s holds key shard (rank - s) mod world; contiguous causal ranks see
+    # s = 0..rank, every other case sees every step
+    return rank if (causal and layout == "contiguous") else world - 1
+
+
+def forward_program(q, k, v, causal: bool, scale: float, rank: int, world: int, ops=None,
+                    layout: str = "contiguous"):
+    """Rank `rank`'s forward: returns (O bf16, LSE fp32) of its query shard.
+    Step 0 is the rank's own key shard, where every query row sees at least
+    its own key, so the first partial result folded in has a finite LSE."""
     ops = ops or CudaOps()
     B, H, n, d = q.shape
     o_acc = torch.empty((B, H, n, d), dtype=torch.float32, device=q.device)
@@ -115,15 +145,16 @@ def forward_program(q, k, v, causal: bool, scale: float, rank: int, world: int, 
     # two buffers of our own (one while only two ranks rotate).
     bufs = [(torch.empty_like(k), torch.empty_like(v)) for _ in range(min(2, world - 1))]
     cur = (k, v)
-    last = _last_visible_step(causal, rank, world)
+    last = _last_visible_step(causal, layout, rank, world)
     first = True
     for s in range(world):
         shard = (rank - s) % world
         if s < world - 1:
             nxt = bufs[s % 2]
             yield ("start", list(cur), list(nxt))
-        if _visible(causal, rank, shard):
-            o_p, l_p = ops.fwd(q, cur[0], cur[1], causal and shard == rank, scale)
+        mask = pair_mask(causal, layout, rank, shard)
+        if mask is not None:
+            o_p, l_p = ops.fwd(q, cur[0], cur[1], mask, scale)
             ops.merge(o_acc, lse_acc, o_p, l_p, o_out if s == last else None, first)
             first = False
         if s < world - 1:
@@ -133,7 +164,7 @@ def forward_program(q, k, v, causal: bool, scale: float, rank: int, world: int, 
 
 
 def backward_program(q, k, v, o, lse, dO, causal: bool, scale: float, rank: int, world: int,
-                     ops=None):
+                     ops=None, layout: str = "contiguous"):
     """Rank `rank`'s backward: returns (dQ, dK, dV) bf16 of its shards, given
     its query shard's final O and LSE (from forward_program)."""
     ops = ops or CudaOps()
@@ -149,9 +180,9 @@ def backward_program(q, k, v, o, lse, dO, causal: bool, scale: float, rank: int,
         if s < world - 1:
             kv_n = bufs[s % 2]
             yield ("start", list(kv), list(kv_n))
-        if _visible(causal, rank, shard):
-            ops.bwd_accumulate(ws, q, kv[0], kv[1], dO, acc[0], acc[1],
-                               causal and shard == rank, scale)
+        mask = pair_mask(causal, layout, rank, shard)
+        if mask is not None:
+            ops.bwd_accumulate(ws, q, kv[0], kv[1], dO, acc[0], acc[1], mask, scale)
         if world > 1:
             # the accumulators belong to key shard `shard`: pass them on; after
             # `world` rotations each is back with its owner
@@ -239,21 +270,37 @@ def run_local(programs):
         reqs = nxt
 
 
-def local_ring_attention(q, k, v, dO, causal: bool, scale: float, world: int, ops=None):
+def local_ring_attention(q, k, v, dO, causal: bool, scale: float, world: int, ops=None,
+                         layout: str = "contiguous"):
     """Forward and backward of attention over the whole [B, H, N, d] inputs,
     computed as a ring of `world` virtual ranks on this device (N divisible by
-    world).  Returns (O, LSE, dQ, dK, dV) for the whole sequence."""
+    world), the sequence laid out over the ranks as `layout` says.  `ops` is
+    one ops object for every rank, or a list of one per rank.  Returns (O,
+    LSE, dQ, dK, dV) for the whole sequence."""
     N = q.shape[2]
     if N % world:
         raise ValueError("sequence length must be divisible by the ring size")
+    if layout not in LAYOUTS:
+        raise ValueError(f"unknown ring layout {layout!r}")
     n = N // world
-    sl = [slice(r * n, (r + 1) * n) for r in range(world)]
+    if layout == "striped":
+        sl = [slice(r, N, world) for r in range(world)]
+    else:
+        sl = [slice(r * n, (r + 1) * n) for r in range(world)]
+    per_rank = ops if isinstance(ops, (list, tuple)) else [ops] * world
     shard = lambda t, r: t[:, :, sl[r]].contiguous()  # noqa: E731
     fwd = run_local([forward_program(shard(q, r), shard(k, r), shard(v, r), causal, scale, r,
-                                     world, ops) for r in range(world)])
+                                     world, per_rank[r], layout) for r in range(world)])
     bwd = run_local([backward_program(shard(q, r), shard(k, r), shard(v, r), fwd[r][0],
-                                      fwd[r][1], shard(dO, r), causal, scale, r, world, ops)
-                     for r in range(world)])
-    cat = lambda xs: torch.cat(xs, dim=2)  # noqa: E731
-    return (cat([f[0] for f in fwd]), cat([f[1] for f in fwd]), cat([b[0] for b in bwd]),
-            cat([b[1] for b in bwd]), cat([b[2] for b in bwd]))
+                                      fwd[r][1], shard(dO, r), causal, scale, r, world,
+                                      per_rank[r], layout) for r in range(world)])
+
+    def gather(parts):
+        out = torch.empty(parts[0].shape[:2] + (N,) + parts[0].shape[3:], dtype=parts[0].dtype,
+                          device=parts[0].device)
+        for r, part in enumerate(parts):
+            out[:, :, sl[r]] = part
+        return out
+
+    return tuple(gather([res[i] for res in part]) for part, i in
+                 ((fwd, 0), (fwd, 1), (bwd, 0), (bwd, 1), (bwd, 2)))

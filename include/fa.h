@@ -65,7 +65,11 @@ typedef enum {
  *   o        [B,H,N,d] bf16, written: O_i = sum_j P_ij v_j.
  *   lse      [B,H,N] fp32, written: LSE_i = ln sum_{j visible} exp(scale q_i.k_j)
  *            (natural log), the statistic fa_bwd consumes.
- *   causal   0 or 1.  scale: multiplies Q K^T (commonly 1/sqrt(d)).
+ *   causal   0: none; 1: key j visible to query i iff j <= i; 2: iff j < i
+ *            (the causal mask without its diagonal, for the pairs of a
+ *            striped ring whose key shard comes later in the sequence; row 0
+ *            then sees no key and gets O = 0, LSE = -inf).
+ *   scale    multiplies Q K^T (commonly 1/sqrt(d)).
  * Cites: FlashAttention-2 abstract (exact attention, tiled, sequence-parallel);
  * iplexlaw blog, "Tiling preserves the attention calculation" (online softmax).
  * Errors: FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_MISALIGNED,
@@ -154,10 +158,15 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *   workspace         device buffer of >= fa_bwd_workspace_size(B,H,N,d)
  *                     bytes, 256-byte aligned; contents need no
  *                     initialisation and are clobbered.
+ * causal as for fa_fwd (0, 1 or 2).
  * Three launches on `stream`: preprocess (D, log2 LSE, zero dQ accumulator),
  * the main kernel (one CTA per key block; recomputes P from LSE; dK, dV per
  * key block; dQ by fp32 reduction), and the dQ conversion to bf16.
  * dQ is not bitwise deterministic (fp32 reduction order varies); dK and dV are.
+ * Cites: iplexlaw blog, "Tiling preserves the attention calculation" (gradient
+ * comparisons within tolerances) and "Why long inputs put pressure on memory"
+ * (the N x N matrices are not stored, so P is recomputed); the gradient
+ * formulas themselves are not on the pages (textbook softmax calculus).
  * Errors: as fa_fwd, plus FA_ERR_INVALID_ARG when the workspace is too small.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o,
@@ -231,7 +240,8 @@ fa_status fa_lse_merge(float* o_acc, float* lse_acc, const void* o_part,
  * of the query rows (over all key shards), calling it once per key/value
  * shard accumulates dQ (in the workspace) and each shard's dK, dV exactly as
  * the gradient over the union of the shards; fa_bwd_dq_convert then yields
- * dQ.  Other arguments and errors as fa_bwd_main.
+ * dQ.  causal 0, 1 or 2 as for fa_fwd.  Other arguments and errors as
+ * fa_bwd_main.
  */
 fa_status fa_bwd_main_accumulate(const void* q, const void* k, const void* v,
                                  const void* dO, float* dk_acc, float* dv_acc,
@@ -328,6 +338,7 @@ fa_status fa_decode_split_plan(int B, int H, int Nq, int Nk, int d,
  * current device's error word.  Returns FA_ERR_TIMEOUT if a kernel's bounded
  * pipeline wait ran out since the last call, FA_ERR_CUDA if the stream
  * reports a CUDA error, FA_OK otherwise.
+ * Cites: not on the pages (failure reporting of this library).
  */
 fa_status fa_get_device_error(void* stream);
 
@@ -340,10 +351,12 @@ fa_status fa_get_device_error(void* stream);
  * following fa_get_device_error(stream) returns FA_ERR_TIMEOUT (and clears
  * the word); the context stays usable.  Errors: FA_ERR_INVALID_ARG for a
  * limit out of range, FA_ERR_UNSUPPORTED / FA_ERR_CUDA as for fa_fwd.
+ * Cites: not on the pages (a test hook of this library's failure path).
  */
 fa_status fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
 
-/* fa_strerror -- static, human-readable name of a status. */
+/* fa_strerror -- static, human-readable name of a status.
+ * Cites: not on the pages. */
 const char* fa_strerror(fa_status status);
 
 #ifdef __cplusplus

@@ -14,8 +14,21 @@ def _np(t):
 
 
 class OracleOps:
+    """`causal` is the library's mask argument: 0 none, 1 key j visible to
+    query i iff j <= i, 2 iff j < i.  Mode 2 is the causal attention of
+    queries 1..n-1 over keys 0..n-2 (query i sees keys j <= i - 1), with row 0
+    seeing no key (O = 0, LSE = -inf; it adds nothing to any gradient)."""
+
     def fwd(self, q, k, v, causal, scale):
-        o, lse = oracle.ref_fwd(_np(q), _np(k), _np(v), causal, scale)
+        if causal == 2:
+            q, k, v = _np(q), _np(k), _np(v)
+            o = np.zeros(q.shape)
+            lse = np.full(q.shape[:3], -np.inf)
+            if q.shape[2] > 1:
+                o[:, :, 1:], lse[:, :, 1:] = oracle.ref_fwd(q[:, :, 1:], k[:, :, :-1],
+                                                            v[:, :, :-1], True, scale)
+            return torch.from_numpy(o), torch.from_numpy(lse)
+        o, lse = oracle.ref_fwd(_np(q), _np(k), _np(v), bool(causal), scale)
         return torch.from_numpy(o), torch.from_numpy(lse)
 
     def merge(self, o_acc, lse_acc, o_part, lse_part, o_out, init):
@@ -33,8 +46,16 @@ class OracleOps:
                 "dq": np.zeros(tuple(o.shape))}
 
     def bwd_accumulate(self, ws, q, k, v, dO, dk_acc, dv_acc, causal, scale):
-        dq, dk, dv = oracle.ref_grads_given_stats(_np(q), _np(k), _np(v), _np(dO), ws["lse"],
-                                                  ws["D"], causal, scale)
+        if causal == 2:
+            q, k, v, dO = _np(q), _np(k), _np(v), _np(dO)
+            dq, dk, dv = np.zeros(q.shape), np.zeros(q.shape), np.zeros(q.shape)
+            if q.shape[2] > 1:
+                dq[:, :, 1:], dk[:, :, :-1], dv[:, :, :-1] = oracle.ref_grads_given_stats(
+                    q[:, :, 1:], k[:, :, :-1], v[:, :, :-1], dO[:, :, 1:],
+                    ws["lse"][:, :, 1:], ws["D"][:, :, 1:], True, scale)
+        else:
+            dq, dk, dv = oracle.ref_grads_given_stats(_np(q), _np(k), _np(v), _np(dO),
+                                                      ws["lse"], ws["D"], bool(causal), scale)
         ws["dq"] += dq
         dk_acc.copy_(torch.from_numpy(_np(dk_acc) + dk))
         dv_acc.copy_(torch.from_numpy(_np(dv_acc) + dv))

@@ -71,7 +71,8 @@ FAKE = 1 << 20  # aligned, never dereferenced: every case fails validation first
     (dict(scale=0.0), fa.FA_ERR_INVALID_ARG),
     (dict(scale=float("nan")), fa.FA_ERR_INVALID_ARG),
     (dict(scale=float("inf")), fa.FA_ERR_INVALID_ARG),
-    (dict(causal=2), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=3), fa.FA_ERR_INVALID_ARG),
+    (dict(causal=-1), fa.FA_ERR_INVALID_ARG),
     (dict(k=FAKE + 2), fa.FA_ERR_MISALIGNED),
     (dict(o=FAKE + 8), fa.FA_ERR_MISALIGNED),
 ])
@@ -89,6 +90,7 @@ def test_fwd_rejects_bad_arguments(lib, kwargs, status):
     (dict(d=32), fa.FA_ERR_UNSUPPORTED),
     (dict(dq=FAKE + 4), fa.FA_ERR_MISALIGNED),
     (dict(workspace=FAKE + 16), fa.FA_ERR_MISALIGNED),
+    (dict(causal=3), fa.FA_ERR_INVALID_ARG),
 ])
 def test_bwd_rejects_bad_arguments(lib, kwargs, status):
     args = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, lse=FAKE, dO=FAKE, dq=FAKE,

@@ -1,12 +1,13 @@
 """Backward parity on the GPU: dQ, dK, dV from the CUDA path (through the C
-ABI) against the oracle's analytic fp64 gradients on the same inputs."""
+ABI) against the oracle's analytic fp64 gradients on the same inputs.  The
+benchmark sweep's shapes are in test_sweep_parity.py."""
 import pytest
 import torch
 
 import exact_attention_109_b200 as fa
 from exact_attention_109_b200.inputs import default_scale
-from parity_util import (check_backward_causal_tail, check_backward_heads,
-                         check_backward_sampled, gpu_inputs, run_backward, run_forward)
+from parity_util import (check_backward_causal_tail, check_backward_heads, gpu_inputs,
+                         run_backward, run_forward)
 
 pytestmark = pytest.mark.gpu
 
@@ -35,42 +36,11 @@ def test_many_heads(causal, d):
     check_backward_heads(host, dq, dk, dv, causal, scale, range(15))
 
 
-@pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("causal", [False, True])
-def test_whole_heads_2048(causal, d):
-    """The fwd+bwd sweep at N=2048 (B=8, width 2048): two whole heads."""
-    B, H = 8, 2048 // d
-    host, dq, dk, dv, scale = _fwd_bwd(B, H, 2048, d, causal, seed=2)
-    check_backward_heads(host, dq, dk, dv, causal, scale, [0, B * H - 1])
-
-
-@pytest.mark.parametrize("N", [4096, 16384])
-@pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("causal", [False, True])
-def test_sweep_sampled(N, d, causal):
-    B, H = 16384 // N, 2048 // d
-    host, dq, dk, dv, scale = _fwd_bwd(B, H, N, d, causal, seed=2)
-    check_backward_sampled(host, dq, dk, dv, causal, scale, [B * H - 1], 32)
-
-
-def test_bench_workload_sampled():
-    """The benchmark's step at full size: B=2 H=16 N=8192 d=128 causal, the
-    same seeded inputs, sampled rows of the first and last heads."""
-    host, dq, dk, dv, scale = _fwd_bwd(2, 16, 8192, 128, True, seed=2)
-    check_backward_sampled(host, dq, dk, dv, True, scale, [0, 31], 32)
-
-
 def test_long_sequence_sampled():
     """B=1 H=16 N=65536 d=128 causal: dQ rows anywhere in two heads, dK/dV
     rows among the last 512 keys."""
     host, dq, dk, dv, scale = _fwd_bwd(1, 16, 65536, 128, True, seed=3)
     check_backward_causal_tail(host, dq, dk, dv, scale, [0, 15], 16, 512)
-
-
-def test_row_scaled_gpt_layer():
-    """GPT layer (a): B=8, N=2048, H=16, d=128, causal, row-scaled Q/K/V."""
-    host, dq, dk, dv, scale = _fwd_bwd(8, 16, 2048, 128, True, seed=4, dist="row_scaled")
-    check_backward_heads(host, dq, dk, dv, True, scale, [0, 127])
 
 
 def test_large_scale_relative():
@@ -112,3 +82,38 @@ def test_workspace_too_small_is_rejected():
                    lse.data_ptr(), dev["dO"].data_ptr(), q.data_ptr(), q.data_ptr(),
                    q.data_ptr(), 1, 1, 256, 64, 0, 0.125, ws.data_ptr(), need - 256)
     assert st == fa.FA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 2, 127, 128, 129, 300, 640])
+def test_strict_causal_mask(N, d):
+    """causal = 2: key j visible to query i iff j < i (the striped ring's
+    pairs with a later key shard).  Row 0 sees no key: O = 0, LSE = -inf, and
+    it adds nothing to any gradient.  For rows i >= 1 the result is causal
+    attention of queries 1..N-1 over keys 0..N-2 (query i sees keys
+    j <= i - 1), which the oracle computes as it is; the last key is seen by
+    no query, so its dK and dV are 0."""
+    import numpy as np
+    import oracle
+    from exact_attention_109_b200.inputs import to_f64
+    from parity_util import Check
+    scale = default_scale(d)
+    host, dev = gpu_inputs(2, 3, N, d, seed=400 + N + d, with_dout=True)
+    o, lse = run_forward(dev, 2, scale)
+    dq, dk, dv = run_backward(dev, o, lse, 2, scale)
+    o, lse, dq, dk, dv = (to_f64(t.cpu()) for t in (o, lse, dq, dk, dv))
+    assert np.all(o[:, :, 0] == 0) and np.all(lse[:, :, 0] == -np.inf)
+    assert np.all(dq[:, :, 0] == 0) and np.all(dk[:, :, N - 1] == 0) and np.all(dv[:, :, N - 1] == 0)
+    if N == 1:
+        return
+    q, k, v, dO = (to_f64(host[x]) for x in ("q", "k", "v", "dO"))
+    sq, sk, sv, sdo = q[:, :, 1:], k[:, :, :-1], v[:, :, :-1], dO[:, :, 1:]
+    o_ref, lse_ref = oracle.ref_fwd(sq, sk, sv, True, scale)
+    rq, rk, rv, _ = oracle.ref_bwd(sq, sk, sv, sdo, True, scale)
+    c = Check()
+    c.o(o[:, :, 1:], o_ref)
+    c.lse(lse[:, :, 1:], lse_ref)
+    c.grad("dq", dq[:, :, 1:], rq)
+    c.grad("dk", dk[:, :, :-1], rk)
+    c.grad("dv", dv[:, :, :-1], rv)
+    c.done()

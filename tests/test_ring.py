@@ -11,8 +11,7 @@ import oracle
 import exact_attention_109_b200 as fa
 from exact_attention_109_b200 import ring
 from exact_attention_109_b200.inputs import attention_inputs, default_scale, to_f64
-from parity_util import (TOL_GRAD_MAX, TOL_LSE_MAX, TOL_O_MAX, TOL_O_REL_L2, max_abs, max_excess,
-                         rel_l2)
+from parity_util import Check, max_abs, max_excess
 
 pytestmark = pytest.mark.gpu
 
@@ -85,37 +84,34 @@ def _check_whole(host, got, causal, scale):
     o_ref, lse_ref = oracle.ref_fwd(*args, causal, scale)
     dq_ref, dk_ref, dv_ref, _ = oracle.ref_bwd(*args, to_f64(host["dO"]), causal, scale)
     o, lse, dq, dk, dv = got
-    og = to_f64(o.cpu())
-    res = {"o_excess": max_excess(og, o_ref), "o_rel_l2": rel_l2(og, o_ref),
-           "lse": max_abs(lse.cpu().double().numpy(), lse_ref)}
+    c = Check()
+    c.o(to_f64(o.cpu()), o_ref)
+    c.lse(lse.cpu().double().numpy(), lse_ref)
     for name, g, r in (("dq", dq, dq_ref), ("dk", dk, dk_ref), ("dv", dv, dv_ref)):
-        res[name] = max_excess(to_f64(g.cpu()), r)
-    assert res["o_excess"] <= TOL_O_MAX, res
-    assert res["o_rel_l2"] <= TOL_O_REL_L2, res
-    assert res["lse"] <= TOL_LSE_MAX, res
-    for name in ("dq", "dk", "dv"):
-        assert res[name] <= TOL_GRAD_MAX, res
-    return res
+        c.grad(name, to_f64(g.cpu()), r)
+    return c.done()
 
 
+@pytest.mark.parametrize("layout", ring.LAYOUTS)
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("world,N", [(1, 384), (2, 512), (3, 600), (4, 1024), (8, 1024)])
-def test_local_ring_matches_whole_sequence(world, N, causal, d):
+def test_local_ring_matches_whole_sequence(world, N, causal, d, layout):
     scale = default_scale(d)
     host = attention_inputs(1, 2, N, d, seed=world * 100 + N + d, with_dout=True)
     q, k, v, dO = (host[x].cuda() for x in ("q", "k", "v", "dO"))
-    got = ring.local_ring_attention(q, k, v, dO, causal, scale, world)
+    got = ring.local_ring_attention(q, k, v, dO, causal, scale, world, layout=layout)
     assert fa.fa_get_device_error() == fa.FA_OK
     _check_whole(host, got, causal, scale)
 
 
-def test_local_ring_long_sequence():
+@pytest.mark.parametrize("layout", ring.LAYOUTS)
+def test_local_ring_long_sequence(layout):
     """4 virtual ranks of 2048 tokens (N = 8192), whole tensors checked."""
     d, causal = 128, True
     scale = default_scale(d)
     host = attention_inputs(1, 2, 8192, d, seed=9, with_dout=True)
     q, k, v, dO = (host[x].cuda() for x in ("q", "k", "v", "dO"))
-    got = ring.local_ring_attention(q, k, v, dO, causal, scale, 4)
+    got = ring.local_ring_attention(q, k, v, dO, causal, scale, 4, layout=layout)
     assert fa.fa_get_device_error() == fa.FA_OK
     _check_whole(host, got, causal, scale)
