@@ -118,11 +118,18 @@ KERNEL_SOURCES = {
 }
 
 
+# Files besides the kernel's own that decide what it does: the PTX helpers
+# (descriptors, MMA and copy wrappers) and the host code that sets its launch.
+SHARED_SOURCES = ("sm100_ptx.cuh", "fa_api.cu")
+
+
 def kernel_sources_hash(kernel: str) -> str:
-    """Hash of the source file that holds the kernel's code."""
-    path = os.path.join(ROOT, "exact_attention_109_b200", "csrc", KERNEL_SOURCES[kernel])
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the kernel's own source file and of the shared sources above."""
+    h = hashlib.sha256()
+    for name in (KERNEL_SOURCES[kernel],) + SHARED_SOURCES:
+        with open(os.path.join(ROOT, "exact_attention_109_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str):
@@ -213,10 +220,11 @@ class ClockSampler:
 def oracle_sample(w, seconds: float, seed: int = 0):
     """Time the fp64 oracle on sampled rows of head 0 of the workload.
 
-    Per-row softmax statistics (LSE_i, D_i) of the head are computed once,
-    untimed; each timed pass then produces O, LSE and dQ for R query rows and
-    dK, dV for R key rows, i.e. R/N of the head's outputs, credited R/N of the
-    head's fwd+bwd FLOPs.  R is sized so one pass takes about `seconds`.
+    Each timed pass first computes the per-row softmax statistics (LSE_i, D_i)
+    of the whole head, which every dK/dV row needs, and then O, LSE and dQ for
+    R query rows and dK, dV for R key rows, i.e. R/N of the head's outputs,
+    credited R/N of the head's fwd+bwd FLOPs (the statistics pass is timed
+    but earns no extra credit).  R is sized so one pass takes about `seconds`.
     Returns (run(R) -> seconds, R, cores, flops_per_pass(R)).
     """
     import numpy as np
@@ -227,7 +235,6 @@ def oracle_sample(w, seconds: float, seed: int = 0):
     q, k, v, dO = (to_f64(inp[x])[0, 0] for x in ("q", "k", "v", "dO"))
     scale = default_scale(w["d"])
     causal = w["causal"]
-    lse, D = oracle.ref_head_stats(q, k, v, dO, causal, scale)
     rng = np.random.default_rng(seed)
     N = w["N"]
     head = dict(w, B=1, H=1)
@@ -236,6 +243,7 @@ def oracle_sample(w, seconds: float, seed: int = 0):
     def run(R):
         rows = np.sort(rng.choice(N, size=R, replace=False))
         t0 = time.perf_counter()
+        lse, D = oracle.ref_head_stats(q, k, v, dO, causal, scale)
         oracle.ref_fwd_rows(q, k, v, rows, causal, scale)
         oracle.ref_dq_rows(q, k, v, dO, rows, causal, scale)
         oracle.ref_dkdv_rows(q, k, v, dO, lse, D, rows, causal, scale)
@@ -243,7 +251,9 @@ def oracle_sample(w, seconds: float, seed: int = 0):
 
     r0 = min(N, 256)
     t = run(r0)
-    R = int(min(N, max(8, math.ceil(r0 * seconds / max(t, 1e-6)))))
+    t_stats = run(1)
+    per_row = max(t - t_stats, 1e-6) / r0
+    R = int(min(N, max(8, math.ceil((seconds - t_stats) / per_row))))
     return run, R, oracle.num_threads(), (lambda r: per_head * r / N)
 
 
@@ -281,7 +291,7 @@ def reference_arm(args, w, wname):
     value = credit(R) * steps / total / 1e12
     sample = (f"{R} of {w['N']} query rows (O, LSE, dQ) and key rows (dK, dV) of one "
               f"head per step, credited {R}/{w['N']} of the head's fwd+bwd FLOPs; "
-              f"per-row LSE/D statistics precomputed untimed")
+              f"each step also recomputes the head's per-row LSE/D statistics (timed)")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": steps, "warmup": warmup,
@@ -323,10 +333,15 @@ def job_throughput(flops_per_rank_step: float, steps: int, world: int,
 
 
 def workload_config(w, wname):
-    return {"workload": wname, "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"],
+    bh, N, d = w["B"] * w["H"], w["N"], w["d"]
+    n_pad = (N + 127) // 128 * 128
+    # q, k, v, o, dO, dq, dk, dv bf16 + LSE, and the fp32 workspace
+    working_set = 8 * bh * N * d * 2 + bh * N * 4 + bh * n_pad * (d + 2) * 4
+    return {"workload": wname, "B": w["B"], "H": w["H"], "N": N, "d": d,
             "causal": w["causal"], "inputs": w["dist"], "pass": "fwd+bwd",
-            "global_batch": w["B"], "seq_len": w["N"],
-            "parallelism": "independent head shards per GPU"}
+            "global_batch": w["B"], "seq_len": N,
+            "parallelism": "independent head shards per GPU",
+            "l2": f"no flush: per-step working set {working_set / 1e6:.0f} MB > 126 MB L2"}
 
 
 # ---------------------------------------------------------------- GPU arm
@@ -534,15 +549,20 @@ def gpu_arm(args, w, wname):
                "sample": (f"oracle ref_fwd + ref_bwd on {heads} whole heads of the "
                           f"workload (N={N}, d={d}, causal={causal}), {tcpu:.1f} s")}
 
+    # ---- the rest of the pages' sweep, measured in the same run (one GPU)
+    sweep = None
+    if world == 1 and not args.no_sweep:
+        sweep = {"note": "fa_fwd / fa_bwd (three launches) per shape through the C ABI; "
+                         "inputs drawn on the device; every working set exceeds L2",
+                 "shapes": measure_sweep(args.warmup, local)}
+
     clocks = clk.summary()
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": elapsed_max / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(w, wname),
-                       l2=("no flush: per-step working set "
-                           f"{(9 * bh * N * d * 2 + ws_bytes) / 1e6:.0f} MB > 126 MB L2")),
+        "config": workload_config(w, wname),
         "fwd_tflops": fwd_t, "bwd_tflops": bwd_t,
         "frac_of_peak": value / peaks["bf16_tflops"],
         "frac_of_datasheet_bf16": value / DATASHEET_BF16_TFLOPS,
@@ -555,6 +575,7 @@ def gpu_arm(args, w, wname):
                         "neighbouring steps on separate streams"},
         "gpu_launches": len(stages) * K,
         "clocks": clocks,
+        "sweep": sweep,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -1082,64 +1103,103 @@ def bias_arm(args, w, wname):
     return 0
 
 
-def sweep_arm(args):
+SWEEP_CASES = ([(16384 // n, 32 if d == 64 else 16, n, d, c, "normal", 2)
+                for n in (512, 1024, 2048, 4096, 8192, 16384) for d in (64, 128)
+                for c in (False, True)]
+               + [(8, 16, 2048, 128, True, "row_scaled", 4),
+                  (2, 20, 8192, 128, True, "row_scaled", 5),
+                  (1, 16, 65536, 128, True, "normal", 3)])
+
+
+def measure_sweep(warmup: int, device_index: int = 0, min_ms: float = 150.0):
     """The whole kernel sweep of the pages' benchmark on one GPU: the 16k-token
     shapes (B*N = 16384, width 2048) for d = 64 and 128, both masks, the two
     GPT-layer shapes (row-scaled inputs) and the N = 65536 sequence, forward
-    and backward through the public API with preallocated outputs and
-    workspace.  One JSON line per shape (not the benchmark contract's single
-    line): TFLOP/s of the forward, the backward (2.5x the forward's FLOPs)
-    and both, each the median of three CUDA-event-timed runs of ten calls."""
+    and backward through the C ABI (fa_fwd, fa_bwd) with preallocated outputs
+    and workspace, inputs drawn on the device.  Per shape: TFLOP/s of the forward,
+    the backward (2.5x the forward's FLOPs) and both, the forward and backward
+    call times in ms (each the median of three CUDA-event-timed runs of R
+    calls, R chosen so a run lasts at least `min_ms` / 3), and the SM clock
+    sampled during those runs.  Every shape's working set exceeds L2."""
     import numpy as np
     import torch
     import exact_attention_109_b200 as fa
-    from exact_attention_109_b200.inputs import attention_inputs, default_scale
-    torch.cuda.set_device(0)
-    cases = [(16384 // n, 32 if d == 64 else 16, n, d, c, "normal", 2)
-             for n in (512, 1024, 2048, 4096, 8192, 16384) for d in (64, 128)
-             for c in (False, True)]
-    cases += [(8, 16, 2048, 128, True, "row_scaled", 4), (2, 20, 8192, 128, True, "row_scaled", 5),
-              (1, 16, 65536, 128, True, "normal", 3)]
-    for (B, H, N, d, causal, dist, seed) in cases:
-        host = attention_inputs(B, H, N, d, seed=seed, dist=dist, with_dout=True)
-        q, k, v, dO = (host[x].cuda() for x in ("q", "k", "v", "dO"))
+    from exact_attention_109_b200.inputs import attention_inputs_device, default_scale
+    rows = []
+    for (B, H, N, d, causal, dist, seed) in SWEEP_CASES:
+        dev = attention_inputs_device(B, H, N, d, seed, dist=dist)
+        q, k, v, dO = dev["q"], dev["k"], dev["v"], dev["dO"]
         sc = default_scale(d)
         ws = torch.empty(fa.fa_bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device="cuda")
         o = torch.empty_like(q)
         lse = torch.empty(B, H, N, device="cuda")
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+
+        stream = torch.cuda.current_stream().cuda_stream
+        P = {x: t.data_ptr() for x, t in dict(q=q, k=k, v=v, dO=dO, o=o, lse=lse, dq=dq, dk=dk,
+                                             dv=dv, ws=ws).items()}
+        nws = ws.numel()
 
         def fwd():
-            fa.attention_forward(q, k, v, causal, sc, out=o, lse=lse)
+            st = fa.fa_fwd(P["q"], P["k"], P["v"], P["o"], P["lse"], B, H, N, d, causal, sc,
+                           stream)
+            if st != fa.FA_OK:
+                raise fa.FaError(st, "sweep fa_fwd")
 
         def bwd():
-            fa.attention_backward(q, k, v, o, lse, dO, causal, sc, workspace=ws)
+            st = fa.fa_bwd(P["q"], P["k"], P["v"], P["o"], P["lse"], P["dO"], P["dq"], P["dk"],
+                           P["dv"], B, H, N, d, causal, sc, P["ws"], nws, stream)
+            if st != fa.FA_OK:
+                raise fa.FaError(st, "sweep fa_bwd")
 
-        for _ in range(args.warmup):
+        for _ in range(max(3, warmup)):
             fwd()
             bwd()
-        torch.cuda.synchronize()
-        reps = 10 if N <= 16384 else 3
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        ev[0].record()
+        fwd()
+        bwd()
+        ev[1].record()
+        torch.cuda.synchronize()
+        reps = max(3, int(math.ceil(min_ms / 3 / max(ev[0].elapsed_time(ev[1]), 1e-3))))
         tf, tb = [], []
-        for _ in range(3):
-            ev[0].record()
-            for _ in range(reps):
-                fwd()
-            ev[1].record()
-            for _ in range(reps):
-                bwd()
-            ev[2].record()
-            torch.cuda.synchronize()
-            tf.append(ev[0].elapsed_time(ev[1]) / reps)
-            tb.append(ev[1].elapsed_time(ev[2]) / reps)
+        with ClockSampler(device_index) as clk:
+            time.sleep(0.25)
+            for _ in range(3):
+                ev[0].record()
+                for _ in range(reps):
+                    fwd()
+                ev[1].record()
+                for _ in range(reps):
+                    bwd()
+                ev[2].record()
+                torch.cuda.synchronize()
+                tf.append(ev[0].elapsed_time(ev[1]) / reps)
+                tb.append(ev[1].elapsed_time(ev[2]) / reps)
         status = fa.fa_get_device_error()
         if status != fa.FA_OK:
             raise fa.FaError(status, "sweep")
         fl = 4.0 * B * H * N * N * d * (0.5 if causal else 1.0)
         f_ms, b_ms = float(np.median(tf)), float(np.median(tb))
-        print(json.dumps({"B": B, "H": H, "N": N, "d": d, "causal": causal, "inputs": dist,
-                          "fwd_tflops": fl / f_ms / 1e9, "bwd_tflops": 2.5 * fl / b_ms / 1e9,
-                          "fwd_bwd_tflops": 3.5 * fl / (f_ms + b_ms) / 1e9}), flush=True)
+        cl = clk.summary()
+        rows.append({"B": B, "H": H, "N": N, "d": d, "causal": causal, "inputs": dist,
+                     "fwd_tflops": round(fl / f_ms / 1e9, 1),
+                     "bwd_tflops": round(2.5 * fl / b_ms / 1e9, 1),
+                     "fwd_bwd_tflops": round(3.5 * fl / (f_ms + b_ms) / 1e9, 1),
+                     "fwd_ms": round(f_ms, 4), "bwd_ms": round(b_ms, 4), "calls": reps,
+                     "clocks": {"sm_mhz": cl["sm_mhz"], "reasons": cl["reasons"],
+                                "samples": cl["samples"]}})
+        del dev, q, k, v, dO, ws, o, lse, dq, dk, dv
+    return rows
+
+
+def sweep_arm(args):
+    """--sweep: print the sweep, one JSON line per shape (not the benchmark
+    contract's single line)."""
+    import torch
+    torch.cuda.set_device(0)
+    for row in measure_sweep(args.warmup):
+        print(json.dumps(row), flush=True)
     return 0
 
 
@@ -1154,6 +1214,8 @@ def main():
                     + sorted(BIAS_WORKLOADS),
                     default=DEFAULT_WORKLOAD)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="leave the per-shape sweep out of the one-GPU line")
     ap.add_argument("--sweep", action="store_true",
                     help="time the whole shape sweep (one JSON line per shape) and exit")
     args = ap.parse_args()

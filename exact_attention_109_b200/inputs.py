@@ -54,16 +54,26 @@ def attention_inputs(B: int, H: int, N: int, d: int, seed: int,
 
 
 def attention_inputs_device(B: int, H: int, N: int, d: int, seed: int,
-                            device="cuda"):
-    """q, k, v, dO of shape [B,H,N,d], "normal" recipe, drawn directly on the
-    device by a seeded ``torch.Generator`` of that device (in the order q, k,
-    v, dO) -- for shapes whose host-side generation and transfer would take
-    minutes.  The bits differ from ``attention_inputs`` with the same seed;
-    a caller that checks a slice against the oracle copies that slice back."""
+                            device="cuda", dist: str = "normal"):
+    """q, k, v, dO of shape [B,H,N,d], drawn directly on the device by a
+    seeded ``torch.Generator`` of that device (in the order q, k, v, dO; the
+    same recipes as above) -- for shapes whose host-side generation and
+    transfer would take minutes.  The bits differ from ``attention_inputs``
+    with the same seed; a caller that checks a slice against the oracle copies
+    that slice back."""
     gen = torch.Generator(device).manual_seed(int(seed))
     shape = (B, H, N, d)
-    return {name: torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
-            .to(torch.bfloat16) for name in ("q", "k", "v", "dO")}
+    out = {}
+    for name in ("q", "k", "v", "dO"):
+        x = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+        if dist == "row_scaled" and name != "dO":
+            r = torch.rand(shape[:-1] + (1,), generator=gen, device=device,
+                           dtype=torch.float32)
+            x = (x * 0.5) * (0.5 + 1.5 * r)
+        elif dist not in ("normal", "row_scaled"):
+            raise ValueError(f"unknown input distribution {dist!r}")
+        out[name] = x.to(torch.bfloat16)
+    return out
 
 
 def decode_inputs(B: int, H: int, Nq: int, Nk: int, d: int, seed: int,
