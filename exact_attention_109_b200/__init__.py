@@ -19,8 +19,9 @@ from .api import (  # noqa: F401
     fa_bwd_preprocess, fa_bwd_main, fa_bwd_dq_convert,
     fa_bwd_noalloc, FA_BWD_NOALLOC_MAX_WORKSPACE_BYTES, fa_selftest_wait_timeout,
     fa_fwd_decode, fa_decode_workspace_size, fa_decode_split_plan,
-    fa_lse_merge, fa_bwd_main_accumulate, fa_convert_f32_bf16, fa_fwd_qk8,
+    fa_lse_merge, fa_bwd_main_accumulate, fa_convert_f32_bf16, fa_fwd_qk8, fa_fwd_fp8,
     fa_fwd_bias, fa_bwd_bias,
     attention_forward, attention_backward, attention_decode, attention_forward_qk8,
+    attention_forward_fp8,
     attention_forward_bias, attention_backward_bias,
 )

@@ -80,6 +80,8 @@ def library():
     lib.fa_convert_f32_bf16.restype = i
     lib.fa_fwd_qk8.argtypes = [vp, vp, vp, f, f, vp, vp, i, i, i, i, i, f, vp]
     lib.fa_fwd_qk8.restype = i
+    lib.fa_fwd_fp8.argtypes = [vp, vp, vp, f, f, f, vp, vp, i, i, i, i, i, f, vp]
+    lib.fa_fwd_fp8.restype = i
     lib.fa_fwd_bias.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp]
     lib.fa_fwd_bias.restype = i
     lib.fa_bwd_bias.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i,
@@ -189,6 +191,14 @@ def fa_fwd_qk8(q: int, k: int, v: int, q_descale: float, k_descale: float, o: in
     """Raw C call: forward pass with e4m3 Q and K; returns the status."""
     return library().fa_fwd_qk8(q, k, v, float(q_descale), float(k_descale), o, lse, B, H, N,
                                 d, int(causal), float(scale), stream or None)
+
+
+def fa_fwd_fp8(q: int, k: int, v: int, q_descale: float, k_descale: float, v_descale: float,
+               o: int, lse: int, B: int, H: int, N: int, d: int, causal: int, scale: float,
+               stream: int = 0) -> int:
+    """Raw C call with device pointers as integers; returns the status."""
+    return library().fa_fwd_fp8(q, k, v, float(q_descale), float(k_descale), float(v_descale),
+                                o, lse, B, H, N, d, int(causal), float(scale), stream or None)
 
 
 def fa_fwd_bias(q: int, k: int, v: int, bias: int, o: int, lse: int, B: int, H: int, N: int,
@@ -349,6 +359,24 @@ def attention_forward_qk8(q8, k8, v, q_descale: float, k_descale: float, causal:
     s = (stream or torch.cuda.current_stream(v.device)).cuda_stream
     _check(fa_fwd_qk8(_ptr(q8), _ptr(k8), _ptr(v), q_descale, k_descale, _ptr(out), _ptr(lse),
                       B, H, N, d, int(causal), scale, s), "fa_fwd_qk8")
+    return out, lse
+
+
+def attention_forward_fp8(q8, k8, v8, q_descale: float, k_descale: float, v_descale: float,
+                          causal: bool, scale: float, out=None, lse=None, stream=None):
+    """O, LSE = fa_fwd_fp8: q8, k8, v8 CUDA float8_e4m3fn [B,H,N,d] with their
+    per-tensor dequantisation factors; O is bf16."""
+    B, H, N, d = _shape(q8)
+    _require({"q8": q8, "k8": k8, "v8": v8}, (B, H, N, d), torch.float8_e4m3fn, q8.device)
+    if out is None:
+        out = torch.empty((B, H, N, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q8.device)
+    _require({"out": out}, (B, H, N, d), torch.bfloat16, q8.device)
+    _require({"lse": lse}, (B, H, N), torch.float32, q8.device)
+    s = (stream or torch.cuda.current_stream(q8.device)).cuda_stream
+    _check(fa_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(v8), q_descale, k_descale, v_descale, _ptr(out),
+                      _ptr(lse), B, H, N, d, int(causal), scale, s), "fa_fwd_fp8")
     return out, lse
 
 

@@ -13,6 +13,7 @@
 #include "fa.h"
 #include "fa_bwd_kernels.cuh"
 #include "fa_decode_kernel.cuh"
+#include "fa_fwd1_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 #include "fa_merge_kernels.cuh"
 
@@ -151,6 +152,22 @@ fa_status device_setup(int* dev_out, unsigned int** err_out) {
                              fa::FwdTraits<128, true>::NUM_THREADS,
                              fa::FwdTraits<128, true>::REG_BUDGET);
         ok &= prepare_fwd_bias<64>() && prepare_fwd_bias<128>();
+        ok &= prepare_kernel(fa::fa_fwd1_kernel<64, false>, fa::Fwd1Traits<64>::SMEM_BYTES,
+                             fa::Fwd1Traits<64>::NUM_THREADS, fa::Fwd1Traits<64>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd1_kernel<64, true>, fa::Fwd1Traits<64>::SMEM_BYTES,
+                             fa::Fwd1Traits<64>::NUM_THREADS, fa::Fwd1Traits<64>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd1_kernel<128, false>, fa::Fwd1Traits<128>::SMEM_BYTES,
+                             fa::Fwd1Traits<128>::NUM_THREADS, fa::Fwd1Traits<128>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd1_kernel<128, true>, fa::Fwd1Traits<128>::SMEM_BYTES,
+                             fa::Fwd1Traits<128>::NUM_THREADS, fa::Fwd1Traits<128>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd_kernel<128, false, true, false, true>,
+                             fa::FwdTraits<128, true, false, true>::SMEM_BYTES,
+                             fa::FwdTraits<128, true, false, true>::NUM_THREADS,
+                             fa::FwdTraits<128, true, false, true>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd_kernel<128, true, true, false, true>,
+                             fa::FwdTraits<128, true, false, true>::SMEM_BYTES,
+                             fa::FwdTraits<128, true, false, true>::NUM_THREADS,
+                             fa::FwdTraits<128, true, false, true>::REG_BUDGET);
         ok &= prepare_kernel(fa::fa_bwd_main_kernel<64, false, true>,
                              fa::BwdTraits<64>::SMEM_BYTES, fa::BwdTraits<64>::NUM_THREADS,
                              fa::BwdTraits<64>::REG_BUDGET);
@@ -214,14 +231,43 @@ bool encode_bf16(CUtensorMap* map, const void* base, int d, int N, long long bh,
 }
 
 // mb: the bias tensor map (BIAS); other variants get any map, unused.
-template <int D, bool CAUSAL, bool QK8 = false, bool BIAS = false>
+template <int D, bool CAUSAL, bool QK8 = false, bool BIAS = false, bool PV8 = false>
 cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                        const CUtensorMap& mo, const CUtensorMap& mb, const fa::FwdParams& prm,
                        long long bh, cudaStream_t stream) {
-    using T = fa::FwdTraits<D, QK8, BIAS>;
+    using T = fa::FwdTraits<D, QK8, BIAS, PV8>;
     const long long grid = bh * prm.n_qpairs;
-    fa::fa_fwd_kernel<D, CAUSAL, QK8, BIAS><<<static_cast<unsigned>(grid), T::NUM_THREADS,
-                                              T::SMEM_BYTES, stream>>>(mq, mk, mv, mo, mb, prm);
+    fa::fa_fwd_kernel<D, CAUSAL, QK8, BIAS, PV8><<<static_cast<unsigned>(grid), T::NUM_THREADS,
+                                                   T::SMEM_BYTES, stream>>>(mq, mk, mv, mo, mb,
+                                                                            prm);
+    return cudaGetLastError();
+}
+
+// Short sequences run the forward with one query tile per CTA and two CTAs
+// per SM (fa_fwd1_kernel), which hides the fixed cost of each CTA behind the
+// other's work; longer ones use fa_fwd_kernel's two tiles per CTA, which
+// share every K/V block between two tiles.  Measured crossover on a B200
+// (16k tokens per batch): the one-tile kernel wins up to N = 512 at both head
+// dims (+2% d = 128, +7-9% d = 64) and at N = 1024 for causal d = 64 (+5%);
+// from N = 1024 on it loses up to 15% at d = 128.  FA_FWD1_MAX_N overrides
+// the threshold (0: never) for experiments.
+#ifndef FA_FWD1_MAX_N
+#define FA_FWD1_MAX_N -1
+#endif
+
+bool use_fwd1(int N, int d, int causal) {
+    if (FA_FWD1_MAX_N >= 0) return N <= FA_FWD1_MAX_N;
+    return N <= 512 || (d == 64 && causal && N <= 1024);
+}
+
+template <int D, bool CAUSAL>
+cudaError_t launch_fwd1(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                        const CUtensorMap& mo, const fa::FwdParams& prm, long long bh,
+                        cudaStream_t stream) {
+    using T = fa::Fwd1Traits<D>;
+    const long long grid = bh * ((prm.N + T::BM - 1) / T::BM);
+    fa::fa_fwd1_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), T::NUM_THREADS, T::SMEM_BYTES,
+                                    stream>>>(mq, mk, mv, mo, prm);
     return cudaGetLastError();
 }
 
@@ -237,6 +283,7 @@ fa::FwdParams fwd_params(float* lse, unsigned int* err, int N, long long bh, int
     prm.bias_batch = 0;
     prm.bias_heads = 0;
     prm.strict = 0;
+    prm.o_scale = 1.0f;
     return prm;
 }
 
@@ -278,6 +325,15 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     prm.strict = causal == 2;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
+    if (use_fwd1(N, d, causal)) {
+        if (d == 64)
+            e = causal ? launch_fwd1<64, true>(mq, mk, mv, mo, prm, bh, s)
+                       : launch_fwd1<64, false>(mq, mk, mv, mo, prm, bh, s);
+        else
+            e = causal ? launch_fwd1<128, true>(mq, mk, mv, mo, prm, bh, s)
+                       : launch_fwd1<128, false>(mq, mk, mv, mo, prm, bh, s);
+        return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    }
     if (d == 64)
         e = causal ? launch_fwd<64, true>(mq, mk, mv, mo, mo, prm, bh, s)
                    : launch_fwd<64, false>(mq, mk, mv, mo, mo, prm, bh, s);
@@ -316,6 +372,43 @@ fa_status fa_fwd_qk8(const void* q, const void* k, const void* v, float q_descal
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const cudaError_t e = causal ? launch_fwd<128, true, true>(mq, mk, mv, mo, mo, prm, bh, s)
                                  : launch_fwd<128, false, true>(mq, mk, mv, mo, mo, prm, bh, s);
+    return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float q_descale,
+                     float k_descale, float v_descale, void* o, float* lse, int B, int H, int N,
+                     int d, int causal, float scale, void* stream) {
+    if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+    fa_status st = check_sizes(B, H, N, d, scale);
+    if (st != FA_OK) return st;
+    if (d != 128) return FA_ERR_UNSUPPORTED;
+    if (!(std::isfinite(q_descale) && q_descale > 0.f && std::isfinite(k_descale) &&
+          k_descale > 0.f && std::isfinite(v_descale) && v_descale > 0.f))
+        return FA_ERR_INVALID_ARG;
+    const float sl2 = scale * q_descale * k_descale * 1.4426950408889634f;
+    if (!(std::isfinite(sl2) && sl2 > 0.f)) return FA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return FA_ERR_MISALIGNED;
+    if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+    int dev;
+    unsigned int* err;
+    if ((st = device_setup(&dev, &err)) != FA_OK) return st;
+    if (!load_encode()) return FA_ERR_CUDA;
+    const long long bh = static_cast<long long>(B) * H;
+    CUtensorMap mq, mk, mv, mo;
+    if (!encode_3d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
+        !encode_3d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
+        !encode_3d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, d, N, bh, 128, 128) ||
+        !encode_bf16(&mo, o, d, N, bh, 32))
+        return FA_ERR_CUDA;
+    fa::FwdParams prm = fwd_params(lse, err, N, bh, H, sl2);
+    // O = v_descale * sum(w V8) / sum(w), with w the e4m3 weights scaled by
+    // 2^PV8_P_SHIFT (the shift cancels in the ratio).
+    prm.o_scale = v_descale;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e =
+        causal ? launch_fwd<128, true, true, false, true>(mq, mk, mv, mo, mo, prm, bh, s)
+               : launch_fwd<128, false, true, false, true>(mq, mk, mv, mo, mo, prm, bh, s);
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

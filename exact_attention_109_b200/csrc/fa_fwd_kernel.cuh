@@ -36,11 +36,18 @@ namespace fa {
 // kind::f8f6f4 MMA at twice the bf16 rate; P and V stay bf16.
 // BIAS: an additive bf16 score bias b_ij, one [128 x 128] tile per query
 // tile and key block, brought in by TMA.
-template <int D, bool QK8 = false, bool BIAS = false>
+// PV8 (with QK8): V is e4m3 too and O += P V also runs as a kind::f8f6f4
+// MMA: P is scaled by 2^PV8_P_SHIFT and rounded to e4m3 in the softmax
+// (a fixed per-block scale that puts the block's weights in e4m3's normal
+// range), the deferred-rescale threshold drops to 2 (log2 units) so that the
+// scaled weights stay below e4m3's maximum 448, and O is normalised by the
+// sum of the rounded weights the MMA used.
+template <int D, bool QK8 = false, bool BIAS = false, bool PV8 = false>
 struct FwdTraits {
     static_assert(D == 64 || D == 128, "head dim");
     static_assert(!QK8 || D == 128, "e4m3 scores need 128-byte rows (d = 128)");
     static_assert(!(QK8 && BIAS), "one variant at a time");
+    static_assert(!PV8 || QK8, "8-bit P V comes with 8-bit scores");
     static constexpr int BM = 128;                  // query rows per tile
     static constexpr int BN = 128;                  // key rows per block
     static constexpr int TILES = 2;                 // query tiles per CTA
@@ -52,6 +59,15 @@ struct FwdTraits {
     static constexpr int QK_CHUNK_COLS = 128 / QK_ELEM;  // elements per swizzle chunk row
     static constexpr int QK_TILE_BYTES = BM * D * QK_ELEM;
     static constexpr int S_KSTEPS = D * QK_ELEM / 32;    // 32-byte K steps of S = Q K^T
+    static constexpr int V_ELEM = PV8 ? 1 : 2;            // bytes per V element
+    static constexpr int V_CHUNKS = D * V_ELEM / 128;
+    static constexpr int V_CHUNK_COLS = 128 / V_ELEM;
+    static constexpr int V_TILE_BYTES = BN * D * V_ELEM;
+    // K steps of O += P V (32 bytes of P per row each: 16 bf16 or 32 e4m3
+    // keys) and the bytes of V each step advances by.
+    static constexpr int PV_KSTEPS = BN * V_ELEM / 32;
+    static constexpr int PV_KSTEP_BYTES = (32 / V_ELEM) * 128;
+    static constexpr int PV8_P_SHIFT = 6;
     static constexpr int NSLOT = (D == 128) ? (BIAS ? 3 : 4) : 8;
     static constexpr int Q_OFF = 0;
     static constexpr int KV_OFF = Q_OFF + TILES * QK_TILE_BYTES;
@@ -79,8 +95,10 @@ struct FwdTraits {
     static constexpr int REG_BUDGET = 128 * (2 * REG_SOFTMAX + REG_CONTROL);
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC_S = QK8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, 0, 0);
-    static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, D, 0, 1);
-    static constexpr float TAU = 8.0f;  // deferred-rescale threshold (log2 units)
+    static constexpr uint32_t IDESC_PV =
+        PV8 ? idesc_e4m3_f32_bmn(128, D) : idesc_bf16_f32(128, D, 0, 1);
+    // deferred-rescale threshold (log2 units)
+    static constexpr float TAU = PV8 ? 2.0f : 8.0f;
     // The softmax signals P per 64-key half and the PV MMA starts on the
     // first half early.  At d = 64 (softmax-bound) that gains; at d = 128
     // the extra TMEM-store wait in the middle of the softmax costs more.
@@ -99,6 +117,7 @@ struct FwdParams {
     int bias_batch;        // bias varies with the batch index (else shared)
     int bias_heads;        // bias varies with the head index (else shared)
     int strict;            // causal mask without the diagonal: key j visible iff j < i
+    float o_scale;         // PV8: V's dequantisation factor (O = o_scale * P V / l)
 };
 
 // One softmax row over a 128-key block: p = exp2(s * scale*log2(e) - m) in
@@ -157,12 +176,58 @@ __device__ __forceinline__ void softmax_block_exp(const uint32_t (&sr)[4][32], f
     lr += (rs[0] + rs[1]) + (rs[2] + rs[3]);
 }
 
-template <int D, bool CAUSAL, bool QK8 = false, bool BIAS = false>
+// The same for 8-bit P V (PV8): each weight is scaled by 2^shift (added to
+// its exponent) and rounded to e4m3, four per TMEM column over the first 32
+// columns of S; lr sums the rounded scaled weights (what the PV MMA uses), l
+// the fp32 unscaled ones.
+__device__ __forceinline__ void softmax_block_exp8(const uint32_t (&sr)[4][32], float sl2,
+                                                   float m, uint32_t s_tm, float& l, float& lr,
+                                                   int shift) {
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    // exp2(x - m + shift) = 2^shift * p: the scale rides in the exponent
+    const uint64_t negm2 = f2_pack(static_cast<float>(shift) - m, static_cast<float>(shift) - m);
+    uint64_t sum2[2] = {0ull, 0ull};
+    float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+            const int c = 64 * h + 2 * e;
+            const uint64_t x2 = ffma2(f2_pack(__uint_as_float(sr[c >> 5][c & 31]),
+                                              __uint_as_float(sr[(c + 1) >> 5][(c + 1) & 31])),
+                                      sl2x2, negm2);
+            float x0, x1;
+            f2_unpack(x2, x0, x1);
+            float p0, p1;
+            if ((e & 3) == 3) {
+                exp2_fma2(x0, x1, p0, p1);
+            } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+            }
+            sum2[e & 1] = fadd2(sum2[e & 1], f2_pack(p0, p1));
+            const uint16_t q = pack_e4m3x2(p0, p1);
+            add_e4m3x2_to_f32(q, rs[2 * (e & 1)], rs[2 * (e & 1) + 1]);
+            if (e & 1)
+                pk[e >> 1] |= static_cast<uint32_t>(q) << 16;
+            else
+                pk[e >> 1] = q;
+        }
+        tmem_st16(s_tm + 16u * h, pk);
+    }
+    float a0, a1;
+    f2_unpack(fadd2(sum2[0], sum2[1]), a0, a1);
+    l += (a0 + a1) * exp2f(static_cast<float>(-shift));
+    lr += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+}
+
+template <int D, bool CAUSAL, bool QK8 = false, bool BIAS = false, bool PV8 = false>
 __global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                   const __grid_constant__ CUtensorMap tmB, const FwdParams p) {
-    using T = FwdTraits<D, QK8, BIAS>;
+    using T = FwdTraits<D, QK8, BIAS, PV8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
 
@@ -233,10 +298,10 @@ __global__ void __launch_bounds__(384, 1)
                 tma_load_3d(smem + T::Q_OFF + t * T::QK_TILE_BYTES + c * T::CHUNK_BYTES, &tmQ,
                             bar_q, c * T::QK_CHUNK_COLS, q0 + 128 * t, bh);
         for (int h = 0; h < 2; ++h) {  // slots 0 and 1: K and V of iteration 0
-            mbar_arrive_expect_tx(&full[h], h ? T::TILE_BYTES : T::QK_TILE_BYTES);
+            mbar_arrive_expect_tx(&full[h], h ? T::V_TILE_BYTES : T::QK_TILE_BYTES);
             uint8_t* dst = smem + T::KV_OFF + h * T::TILE_BYTES;
-            const int nch = h ? T::CHUNKS : T::QK_CHUNKS;
-            const int ccols = h ? 64 : T::QK_CHUNK_COLS;
+            const int nch = h ? T::V_CHUNKS : T::QK_CHUNKS;
+            const int ccols = h ? T::V_CHUNK_COLS : T::QK_CHUNK_COLS;
             for (int c = 0; c < nch; ++c)
                 tma_load_3d(dst + c * T::CHUNK_BYTES, h ? &tmV : &tmK, &full[h], c * ccols,
                             kv_block(0) * T::BN, bh);
@@ -274,10 +339,10 @@ __global__ void __launch_bounds__(384, 1)
                         ok = false;
                         break;
                     }
-                    mbar_arrive_expect_tx(&full[slot], h ? T::TILE_BYTES : T::QK_TILE_BYTES);
+                    mbar_arrive_expect_tx(&full[slot], h ? T::V_TILE_BYTES : T::QK_TILE_BYTES);
                     uint8_t* dst = smem + T::KV_OFF + slot * T::TILE_BYTES;
-                    const int nch = h ? T::CHUNKS : T::QK_CHUNKS;
-                    const int ccols = h ? 64 : T::QK_CHUNK_COLS;
+                    const int nch = h ? T::V_CHUNKS : T::QK_CHUNKS;
+                    const int ccols = h ? T::V_CHUNK_COLS : T::QK_CHUNK_COLS;
                     for (int c = 0; c < nch; ++c)
                         tma_load_3d(dst + c * T::CHUNK_BYTES, h ? &tmV : &tmK, &full[slot],
                                     c * ccols, kv_block(j) * T::BN, bh);
@@ -356,12 +421,15 @@ __global__ void __launch_bounds__(384, 1)
                 const uint64_t dv0 = sdesc_sw128(v_addr, T::CHUNK_BYTES, 1024);
 #pragma unroll
                 for (int k = k0; k < k1; ++k) {
-                    if (k == 0)
-                        umma_ts(tmem + 256u + D * t, tmem + 128u * t, dv0, T::IDESC_PV,
-                                accumulate ? 1u : 0u);
+                    const uint32_t a = tmem + 128u * t + 8u * k;  // 32 bytes of P per row
+                    const uint64_t b = sdesc_add(dv0, k * T::PV_KSTEP_BYTES);
+                    const uint32_t acc = (k > 0 || accumulate) ? 1u : 0u;
+                    if constexpr (PV8)
+                        umma_ts_f8(tmem + 256u + D * t, a, b, T::IDESC_PV, acc);
+                    else if (k == 0)
+                        umma_ts(tmem + 256u + D * t, a, b, T::IDESC_PV, acc);
                     else
-                        umma_ts_c<true>(tmem + 256u + D * t, tmem + 128u * t + 8u * k,
-                                        sdesc_add(dv0, k * 2048), T::IDESC_PV);
+                        umma_ts_c<true>(tmem + 256u + D * t, a, b, T::IDESC_PV);
                 }
             };
             // PV of tile t for the block whose P has phase `par`: in two
@@ -370,14 +438,14 @@ __global__ void __launch_bounds__(384, 1)
                 if constexpr (T::PSPLIT) {
                     if (!mbar_wait(&p_half[t], par, st)) return false;
                     tc_fence_after();
-                    mma_pv(t, v_addr, acc, 0, T::BN / 32);
+                    mma_pv(t, v_addr, acc, 0, T::PV_KSTEPS / 2);
                     if (!mbar_wait(&p_ready[t], par, st)) return false;
                     tc_fence_after();
-                    mma_pv(t, v_addr, true, T::BN / 32, T::BN / 16);
+                    mma_pv(t, v_addr, true, T::PV_KSTEPS / 2, T::PV_KSTEPS);
                 } else {
                     if (!mbar_wait(&p_ready[t], par, st)) return false;
                     tc_fence_after();
-                    mma_pv(t, v_addr, acc, 0, T::BN / 16);
+                    mma_pv(t, v_addr, acc, 0, T::PV_KSTEPS);
                 }
                 return true;
             };
@@ -541,8 +609,12 @@ __global__ void __launch_bounds__(384, 1)
             m = m_new;
             // A row that has seen no visible key yet (only the strict causal
             // mask's row 0) keeps m = -inf; its weights are exp2(-inf) = 0.
-            softmax_block_exp<T::PSPLIT>(sr, sl2e, m == -INFINITY ? 0.f : m, s_tm, l, lr,
-                                         &p_half[t]);
+            if constexpr (PV8)
+                softmax_block_exp8(sr, sl2e, m == -INFINITY ? 0.f : m, s_tm, l, lr,
+                                   T::PV8_P_SHIFT);
+            else
+                softmax_block_exp<T::PSPLIT>(sr, sl2e, m == -INFINITY ? 0.f : m, s_tm, l, lr,
+                                             &p_half[t]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&p_ready[t]);
@@ -554,7 +626,7 @@ __global__ void __launch_bounds__(384, 1)
             // A row with no visible key (strict causal row 0) keeps m = -inf:
             // O = 0, LSE = -inf.  (Its weights are not all 0 -- the FMA-pipe
             // exp2 returns 2^-126 for -inf -- so lr alone cannot tell.)
-            const float inv_l = m == -INFINITY ? 0.f : 1.0f / lr;
+            const float inv_l = m == -INFINITY ? 0.f : (PV8 ? p.o_scale : 1.0f) / lr;
             const float lse_val = (m + log2f(l)) * 0.6931471805599453f;
             // Stage O (bf16, 128-byte swizzle) in this tile's Q buffer, which
             // no MMA reads any more (e4m3 scores: in the staging region),

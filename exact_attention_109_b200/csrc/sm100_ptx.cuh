@@ -268,6 +268,19 @@ __device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uin
         : "memory");
 }
 
+// D[tmem] (+)= A[tmem] * B[smem desc] for 8-bit float operands (kind::f8f6f4,
+// e4m3 here), fp32 accumulation, K = 32 per call; A K-major in TMEM (four
+// e4m3 values per 32-bit column, the lowest byte first).
+__device__ __forceinline__ void umma_ts_f8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05 async op issued so far by this
 // thread has completed.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
@@ -349,6 +362,11 @@ __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
            | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
+// The same with B MN-major (e4m3 is one of the types that allow it).
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32_bmn(int M, int N) {
+    return idesc_e4m3_f32(M, N) | (1u << 16);
+}
+
 // TMEM load: 32 lanes x 32 bits, 32 consecutive columns per thread.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -413,6 +431,24 @@ __device__ __forceinline__ void add_bf16x2_to_f32(uint32_t pk, float& acc_lo, fl
     asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
         "add.rn.f32.bf16 %0, lo, %0;\n\tadd.rn.f32.bf16 %1, hi, %1;\n\t}"
         : "+f"(acc_lo), "+f"(acc_hi) : "r"(pk));
+}
+
+// Two floats to e4m3 (round to nearest even, saturating at +-448): `lo` in
+// the low byte.
+__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// acc_lo + (low e4m3 byte of `pk`), acc_hi + (high byte): exact widening
+// through f16, fp32 add.
+__device__ __forceinline__ void add_e4m3x2_to_f32(uint16_t pk, float& acc_lo, float& acc_hi) {
+    asm("{\n\t.reg .b32 h2;\n\t.reg .b16 lo, hi;\n\t"
+        "cvt.rn.f16x2.e4m3x2 h2, %2;\n\t"
+        "mov.b32 {lo, hi}, h2;\n\t"
+        "add.rn.f32.f16 %0, lo, %0;\n\tadd.rn.f32.f16 %1, hi, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi) : "h"(pk));
 }
 
 // Two-lane fp32 vectors in one 64-bit register pair (sm_100 f32x2 ops).

@@ -102,6 +102,32 @@ fa_status fa_fwd_qk8(const void* q, const void* k, const void* v,
                      void* stream);
 
 /*
+ * fa_fwd_fp8 -- forward pass with both products in 8-bit floats (the next
+ * step of the low-precision attention on Blackwell tensor cores the pages
+ * cite): Q, K and V are e4m3, S = Q K^T and O += P V both run as
+ * tcgen05.mma kind::f8f6f4.
+ *   q, k, v  [B,H,N,d] e4m3 (OCP FP8 E4M3), read only, with per-tensor
+ *            dequantisation factors q_descale, k_descale, v_descale (finite,
+ *            > 0): the attention is that of the dequantised tensors.
+ *   o        [B,H,N,d] bf16, written; lse as fa_fwd.
+ * P is scaled by 2^6 and rounded to e4m3 in the softmax (the running maximum
+ * is refreshed once a row's scores exceed it by 2 in log2 units, so the
+ * scaled weights stay below e4m3's 448), and O is normalised by the sum of
+ * the rounded weights, so O is an exact convex combination of V rows under
+ * weights that each carry up to 2^-4 relative rounding (2^-3 after
+ * normalising).  LSE uses the unrounded fp32 weights, as in fa_fwd.
+ * Contract, per element, against the definition on the dequantised inputs:
+ *   |O - O_ref| <= 2^-3 * sum_j P_ij |v_j - O_ref,i| + 2^-8 |O_ref| + 4e-3,
+ *   relative L2 of O <= 6e-2, LSE max-abs <= 1e-3.
+ * Supported: d = 128, causal 0 or 1.  Other conventions and errors as
+ * fa_fwd_qk8 (FA_ERR_INVALID_ARG for a descale that is not finite and > 0).
+ */
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v,
+                     float q_descale, float k_descale, float v_descale, void* o,
+                     float* lse, int B, int H, int N, int d, int causal,
+                     float scale, void* stream);
+
+/*
  * Attention with an additive score bias: S_ij = scale * q_i.k_j + b_ij
  * (a prior added to the query-key scores, the "attention with bias" of
  * vision, language and protein-folding models that the pages cite), before
