@@ -58,6 +58,11 @@ QK8_WORKLOADS = {
                                             dist="normal", seed=2),
     "fwd_qk8_sweep_N8192_d128_noncausal": dict(B=2, H=16, N=8192, d=128, causal=False,
                                                dist="normal", seed=2),
+    # fa_fwd_fp8: V in e4m3 too, both products on the 8-bit path
+    "fwd_fp8_sweep_N8192_d128_causal": dict(B=2, H=16, N=8192, d=128, causal=True,
+                                            dist="normal", seed=2, pv8=True),
+    "fwd_fp8_sweep_N8192_d128_noncausal": dict(B=2, H=16, N=8192, d=128, causal=False,
+                                               dist="normal", seed=2, pv8=True),
 }
 
 # Additive score bias (fa_fwd_bias / fa_bwd_bias): 16k tokens, a bias shared
@@ -71,9 +76,12 @@ BIAS_WORKLOADS = {
 # single-sequence shape split into G shards of N/G tokens.
 RING_WORKLOADS = {
     "ring_G4_B1_H16_N65536_d128_causal": dict(B=1, H=16, N=65536, d=128, causal=True,
-                                              dist="normal", seed=3, G=4),
+                                              dist="normal", seed=3, G=4, layout="contiguous"),
+    "ring_G4_B1_H16_N65536_d128_causal_striped": dict(B=1, H=16, N=65536, d=128, causal=True,
+                                                      dist="normal", seed=3, G=4,
+                                                      layout="striped"),
     "ring_G2_B2_H16_N8192_d128_causal": dict(B=2, H=16, N=8192, d=128, causal=True,
-                                             dist="normal", seed=2, G=2),
+                                             dist="normal", seed=2, G=2, layout="contiguous"),
 }
 DEFAULT_WORKLOAD = "fwd_bwd_sweep_N8192_d128_causal"
 
@@ -786,6 +794,35 @@ def decode_arm(args, w, wname):
 # ---------------------------------------------------------------- ring
 
 
+class _TimedRingOps:
+    """The ring's CUDA ops with CUDA events around every call, so that each
+    virtual rank's own device time can be summed."""
+
+    def __init__(self):
+        from exact_attention_109_b200 import ring
+        self._ops = ring.CudaOps()
+        self._events = []
+
+    def _timed(self, name):
+        import torch
+        fn = getattr(self._ops, name)
+
+        def call(*a, **kw):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            out = fn(*a, **kw)
+            e1.record()
+            self._events.append((e0, e1))
+            return out
+        return call
+
+    def __getattr__(self, name):
+        return self._timed(name)
+
+    def total_ms(self):
+        return sum(a.elapsed_time(b) for a, b in self._events)
+
+
 def ring_arm(args, w, wname):
     """G virtual ranks on this GPU (exact_attention_109_b200.ring.run_local):
     one step = the ring forward and backward over the whole sequence, every
@@ -808,8 +845,10 @@ def ring_arm(args, w, wname):
     q, k, v, dO = (host[x].cuda() for x in ("q", "k", "v", "dO"))
     stream = torch.cuda.current_stream()
 
+    layout = w.get("layout", "contiguous")
+
     def step():
-        return ring.local_ring_attention(q, k, v, dO, causal, scale, G)
+        return ring.local_ring_attention(q, k, v, dO, causal, scale, G, layout=layout)
 
     def plain_step():
         o, lse = fa.attention_forward(q, k, v, causal, scale)
@@ -853,13 +892,27 @@ def ring_arm(args, w, wname):
     for _ in range(Ke):
         for x in pin:
             dev[x].copy_(pin[x], non_blocking=True)
-        got = ring.local_ring_attention(dev["q"], dev["k"], dev["v"], dev["dO"], causal, scale, G)
+        got = ring.local_ring_attention(dev["q"], dev["k"], dev["v"], dev["dO"], causal, scale, G,
+                                        layout=layout)
         outs = [t.to("cpu", non_blocking=True) for t in got]
     e1.record(stream)
     torch.cuda.synchronize()
     e2e = flops / (e0.elapsed_time(e1) / Ke * 1e-3) / 1e12
     h2d = sum(t.numel() * t.element_size() for t in pin.values())
     d2h = sum(t.numel() * t.element_size() for t in outs)
+
+    # Per-rank work: the device time of each virtual rank's own kernels (its
+    # pair attention, merges and conversions; rotations excluded).  On G
+    # GPUs with overlapped transfers the slowest rank sets the ring's time,
+    # which is what the layouts differ in under the causal mask.
+    per_rank = {}
+    for lay in ring.LAYOUTS:
+        timers = [_TimedRingOps() for _ in range(G)]
+        ring.local_ring_attention(q, k, v, dO, causal, scale, G, ops=timers, layout=lay)
+        torch.cuda.synchronize()
+        ms = [t.total_ms() for t in timers]
+        per_rank[lay] = {"per_rank_ms": [round(x, 3) for x in ms],
+                         "critical_path_ms": round(max(ms), 3)}
 
     peaks = load_peaks()
     cpu = None
@@ -876,11 +929,13 @@ def ring_arm(args, w, wname):
         "warmup": args.warmup, "ms_per_step": ring_ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(w, wname), **{
-            "G": G, "pass": "ring fwd+bwd",
+            "G": G, "layout": layout, "pass": "ring fwd+bwd",
             "parallelism": f"ring of {G} virtual ranks on one GPU",
             "l2": f"no flush: per-step working set {9 * B * H * N * d * 2 / 1e6:.0f} MB"}),
         "plain_fwd_bwd_tflops": flops / (plain_ms * 1e-3) / 1e12,
         "ring_overhead": ring_ms / plain_ms - 1.0,
+        "layout": layout,
+        "per_rank_work": per_rank,
         "roofline": {"kernel": "whole ring step (fa_fwd, fa_lse_merge, fa_bwd_*)",
                      "bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
@@ -901,7 +956,9 @@ def qk8_arm(args, w, wname):
     dequantised bf16 inputs.  S = QK^T runs at the e4m3 rate and P V at the
     bf16 rate, so the roofline peak is the harmonic mix of the two: half the
     FLOPs at 2x the measured bf16 peak (the nominal e4m3:bf16 ratio of 2),
-    half at 1x, i.e. 4/3 of the bf16 peak."""
+    half at 1x, i.e. 4/3 of the bf16 peak.  With pv8 the workload runs
+    fa_fwd_fp8 instead (V e4m3 too, both products at the e4m3 rate: peak 2x
+    the bf16 one), timed beside fa_fwd_qk8 and fa_fwd."""
     import torch
 
     import exact_attention_109_b200 as fa
@@ -916,28 +973,42 @@ def qk8_arm(args, w, wname):
     host = attention_inputs(B, H, N, d, w["seed"], w["dist"])
     q8, qs = to_e4m3(host["q"])
     k8, ks = to_e4m3(host["k"])
+    pv8 = bool(w.get("pv8"))
+    v8, vs = to_e4m3(host["v"])
     q8d, k8d, v = q8.cuda(), k8.cuda(), host["v"].cuda()
+    v8d = v8.cuda()
     qd = (q8.to(torch.float32) * qs).to(torch.bfloat16).cuda()
     kd = (k8.to(torch.float32) * ks).to(torch.bfloat16).cuda()
+    vd = (v8.to(torch.float32) * vs).to(torch.bfloat16).cuda() if pv8 else v
     o = torch.empty_like(v)
     lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
     s = torch.cuda.current_stream()
 
-    def step():
-        st = fa.fa_fwd_qk8(q8d.data_ptr(), k8d.data_ptr(), v.data_ptr(), qs, ks, o.data_ptr(),
+    def qk8_step():
+        st = fa.fa_fwd_qk8(q8d.data_ptr(), k8d.data_ptr(), vd.data_ptr(), qs, ks, o.data_ptr(),
                            lse.data_ptr(), B, H, N, d, int(causal), scale, s.cuda_stream)
         if st != fa.FA_OK:
             raise fa.FaError(st, "qk8 step")
 
+    def fp8_step():
+        st = fa.fa_fwd_fp8(q8d.data_ptr(), k8d.data_ptr(), v8d.data_ptr(), qs, ks, vs,
+                           o.data_ptr(), lse.data_ptr(), B, H, N, d, int(causal), scale,
+                           s.cuda_stream)
+        if st != fa.FA_OK:
+            raise fa.FaError(st, "fp8 step")
+
+    step = fp8_step if pv8 else qk8_step
+
     def bf16_step():
-        fa.attention_forward(qd, kd, v, causal, scale, out=o, lse=lse)
+        fa.attention_forward(qd, kd, vd, causal, scale, out=o, lse=lse)
 
     for _ in range(args.warmup):
         step()
+        qk8_step()
         bf16_step()
     torch.cuda.synchronize()
     K = args.steps
-    e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
     with ClockSampler(0) as clk:
         time.sleep(0.3)
         torch.cuda.synchronize()
@@ -948,16 +1019,20 @@ def qk8_arm(args, w, wname):
         for _ in range(K):
             bf16_step()
         e[2].record(s)
+        for _ in range(K):
+            qk8_step()
+        e[4].record(s)
         torch.cuda.synchronize()
     if fa.fa_get_device_error() != fa.FA_OK:
-        raise RuntimeError("qk8 timed region: device error")
+        raise RuntimeError("e4m3 timed region: device error")
     ms = e[0].elapsed_time(e[1]) / K
     bf16_ms = e[1].elapsed_time(e[2]) / K
+    qk8_ms = e[2].elapsed_time(e[4]) / K
     flops = fwd_flops(w)
     value = flops / (ms * 1e-3) / 1e12
     # end to end: q8, k8, v in from pinned host memory, O and LSE out
-    pin = [q8.pin_memory(), k8.pin_memory(), host["v"].pin_memory()]
-    dst = [torch.empty_like(q8d), torch.empty_like(k8d), torch.empty_like(v)]
+    pin = [q8.pin_memory(), k8.pin_memory(), (v8 if pv8 else host["v"]).pin_memory()]
+    dst = [torch.empty_like(q8d), torch.empty_like(k8d), torch.empty_like(v8d if pv8 else v)]
     oh = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
     lh = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
     Ke = max(4, min(K, 20))
@@ -965,14 +1040,19 @@ def qk8_arm(args, w, wname):
     for _ in range(Ke):
         for a, b in zip(pin, dst):
             b.copy_(a, non_blocking=True)
-        fa.attention_forward_qk8(dst[0], dst[1], dst[2], qs, ks, causal, scale, out=o, lse=lse)
+        if pv8:
+            fa.attention_forward_fp8(dst[0], dst[1], dst[2], qs, ks, vs, causal, scale, out=o,
+                                     lse=lse)
+        else:
+            fa.attention_forward_qk8(dst[0], dst[1], dst[2], qs, ks, causal, scale, out=o,
+                                     lse=lse)
         oh.copy_(o, non_blocking=True)
         lh.copy_(lse, non_blocking=True)
     e[3].record(s)
     torch.cuda.synchronize()
     e2e = flops / (e[0].elapsed_time(e[3]) / Ke * 1e-3) / 1e12
     peaks = load_peaks()
-    mixed_peak = peaks["bf16_tflops"] * 4.0 / 3.0
+    mixed_peak = peaks["bf16_tflops"] * (2.0 if pv8 else 4.0 / 3.0)
     cpu = None
     if not args.no_cpu_baseline:
         val, tcpu, heads, cores = oracle_whole_heads(w, 20.0)
@@ -982,17 +1062,22 @@ def qk8_arm(args, w, wname):
     print(json.dumps({
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": 1, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "e4m3 QK^T, bf16 PV", "data": "synthetic",
+        "vs_baseline": None, "dtype": "e4m3 QK^T and PV" if pv8 else "e4m3 QK^T, bf16 PV",
+        "data": "synthetic",
         "config": dict(workload_config(w, wname), **{"pass": "fwd", "quant": "per-tensor e4m3 "
-                       "Q, K (descale = amax / 448)",
+                       + ("Q, K, V" if pv8 else "Q, K") + " (descale = amax / 448)",
                        "l2": f"no flush: per-step working set {(2 + 4) * B * H * N * d / 1e6:.0f} MB"}),
         "bf16_fwd_tflops": flops / (bf16_ms * 1e-3) / 1e12,
+        "qk8_fwd_tflops": flops / (qk8_ms * 1e-3) / 1e12,
         "speedup_vs_bf16": bf16_ms / ms,
-        "roofline": {"kernel": "fa_fwd_kernel<128, causal, e4m3>", "bound": "tensor",
+        "roofline": {"kernel": "fa_fwd_kernel<128, causal, e4m3" + (" QK and PV>" if pv8
+                                                                    else " QK>"),
+                     "bound": "tensor",
                      "achieved": value, "peak": mixed_peak, "unit": "TFLOP/s",
                      "frac": value / mixed_peak,
-                     "peak_source": f"{peaks['source']} bf16 burst x 4/3 (half the FLOPs at the "
-                                    f"nominal 2x e4m3 rate)", "traffic": None},
+                     "peak_source": f"{peaks['source']} bf16 burst x " + (
+                         "2 (all FLOPs at the nominal 2x e4m3 rate)" if pv8 else
+                         "4/3 (half the FLOPs at the nominal 2x e4m3 rate)"), "traffic": None},
         "cpu_baseline": cpu,
         "e2e": {"value": e2e, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in pin),
