@@ -448,6 +448,9 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
         const int lg = warp & 3;
         const int r = lg * 32 + lane;
         const int kv_row = j * T::BN + r;
+        // Key rows past N (zero-filled K, V): P = 0, so that a score of 0
+        // against a very negative LSE cannot overflow into dS.
+        const bool row_live = kv_row < N;
         const uint32_t lane_off = static_cast<uint32_t>(lg * 32) << 16;
         const float sl2 = p.scale_log2;
         // Bias and its gradient are read and written straight from / to HBM:
@@ -528,7 +531,7 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
                         arg = fmaf(bv, 1.4426950408889634f, arg);
                     }
                     float x = ex2_approx(fmaf(__uint_as_float(sv[e]), sl2, arg));
-                    if (CAUSAL && e < masked) x = 0.f;
+                    if (!row_live || (CAUSAL && e < masked)) x = 0.f;
                     pr[h] = x;
                     ds[h] = x * (__uint_as_float(dp[e]) - dsv_[h]);
                 }
@@ -711,7 +714,7 @@ cudaError_t launch_bwd_main(int bh, int N, float scale, const BwdWorkspace& ws,
                             void* dbias = nullptr, int H = 1, int bias_batch = 0,
                             int bias_heads = 0, int strict = 0) {
     using T = BwdTraits<D>;
-    BwdParams prm;
+    BwdParams prm{};
     prm.lse2 = ws.lse2;
     prm.dvec = ws.dvec;
     prm.err = err;
