@@ -243,16 +243,22 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     return cudaGetLastError();
 }
 
-// Short sequences run the forward with one query tile per CTA and two CTAs
-// per SM (fa_fwd1_kernel), which hides the fixed cost of each CTA behind the
-// other's work; longer ones use fa_fwd_kernel's two tiles per CTA, which
+// Short sequences run the forward with one query tile at a time per CTA,
+// two persistent CTAs per SM (fa_fwd1_kernel), which hides the fixed cost
+// around each tile; longer ones use fa_fwd_kernel's two tiles per CTA, which
 // share every K/V block between two tiles.  Measured crossover on a B200
-// (16k tokens per batch): the one-tile kernel wins up to N = 512 at both head
-// dims (+2% d = 128, +7-9% d = 64) and at N = 1024 for causal d = 64 (+5%);
-// from N = 1024 on it loses up to 15% at d = 128.  FA_FWD1_MAX_N overrides
-// the threshold (0: never) for experiments.
+// (16k tokens per batch, forward TFLOP/s): the one-tile kernel wins up to
+// N = 512 at both head dims (+9-16% d = 64, +9% d = 128) and at N = 1024 for
+// causal d = 64 (+10%); from N = 1024 on it loses up to 19% at d = 128.
+// FA_FWD1_MAX_N overrides the threshold (0: never) for experiments.
 #ifndef FA_FWD1_MAX_N
 #define FA_FWD1_MAX_N -1
+#endif
+
+// FA_FWD1_CTAS_PER_SM=0 at build time launches one CTA per tile instead of
+// the persistent grid, for comparisons.
+#ifndef FA_FWD1_CTAS_PER_SM
+#define FA_FWD1_CTAS_PER_SM 2
 #endif
 
 bool use_fwd1(int N, int d, int causal) {
@@ -263,9 +269,13 @@ bool use_fwd1(int N, int d, int causal) {
 template <int D, bool CAUSAL>
 cudaError_t launch_fwd1(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                         const CUtensorMap& mo, const fa::FwdParams& prm, long long bh,
-                        cudaStream_t stream) {
+                        int sm_count, cudaStream_t stream) {
     using T = fa::Fwd1Traits<D>;
-    const long long grid = bh * ((prm.N + T::BM - 1) / T::BM);
+    // Persistent: at most two CTAs per SM (the occupancy the kernel is built
+    // for), each walking every grid-th tile.
+    const long long tiles = bh * ((prm.N + T::BM - 1) / T::BM);
+    const long long cap = FA_FWD1_CTAS_PER_SM > 0 ? 2LL * std::max(1, sm_count) : tiles;
+    const long long grid = std::min(tiles, cap);
     fa::fa_fwd1_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), T::NUM_THREADS, T::SMEM_BYTES,
                                     stream>>>(mq, mk, mv, mo, prm);
     return cudaGetLastError();
@@ -327,11 +337,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     cudaError_t e;
     if (use_fwd1(N, d, causal)) {
         if (d == 64)
-            e = causal ? launch_fwd1<64, true>(mq, mk, mv, mo, prm, bh, s)
-                       : launch_fwd1<64, false>(mq, mk, mv, mo, prm, bh, s);
+            e = causal ? launch_fwd1<64, true>(mq, mk, mv, mo, prm, bh, g_dev[dev].sm_count, s)
+                       : launch_fwd1<64, false>(mq, mk, mv, mo, prm, bh, g_dev[dev].sm_count, s);
         else
-            e = causal ? launch_fwd1<128, true>(mq, mk, mv, mo, prm, bh, s)
-                       : launch_fwd1<128, false>(mq, mk, mv, mo, prm, bh, s);
+            e = causal ? launch_fwd1<128, true>(mq, mk, mv, mo, prm, bh, g_dev[dev].sm_count, s)
+                       : launch_fwd1<128, false>(mq, mk, mv, mo, prm, bh, g_dev[dev].sm_count, s);
         return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
     }
     if (d == 64)
