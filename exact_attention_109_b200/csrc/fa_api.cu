@@ -248,7 +248,7 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 // around each tile; longer ones use fa_fwd_kernel's two tiles per CTA, which
 // share every K/V block between two tiles.  Measured crossover on a B200
 // (16k tokens per batch, forward TFLOP/s): the one-tile kernel wins up to
-// N = 512 at both head dims (+9-16% d = 64, +9% d = 128) and at N = 1024 for
+// N = 512 at both head dims (+16-25% d = 64, +9% d = 128) and at N = 1024 for
 // causal d = 64 (+10%); from N = 1024 on it loses up to 19% at d = 128.
 // FA_FWD1_MAX_N overrides the threshold (0: never) for experiments.
 #ifndef FA_FWD1_MAX_N
