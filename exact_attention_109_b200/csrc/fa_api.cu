@@ -11,6 +11,7 @@
 #include <mutex>
 
 #include "fa.h"
+#include "fa_bwd64_kernel.cuh"
 #include "fa_bwd_kernels.cuh"
 #include "fa_decode_kernel.cuh"
 #include "fa_fwd1_kernel.cuh"
@@ -143,6 +144,10 @@ fa_status device_setup(int* dev_out, unsigned int** err_out) {
                              fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
         ok &= prepare_kernel(fa::fa_bwd_main_kernel<128, true>, fa::BwdTraits<128>::SMEM_BYTES,
                              fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_bwd_main64_kernel<false>, fa::Bwd64Traits::SMEM_BYTES,
+                             fa::Bwd64Traits::NUM_THREADS, fa::Bwd64Traits::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_bwd_main64_kernel<true>, fa::Bwd64Traits::SMEM_BYTES,
+                             fa::Bwd64Traits::NUM_THREADS, fa::Bwd64Traits::REG_BUDGET);
         ok &= prepare_kernel(fa::fa_fwd_kernel<128, false, true>,
                              fa::FwdTraits<128, true>::SMEM_BYTES,
                              fa::FwdTraits<128, true>::NUM_THREADS,
@@ -500,6 +505,13 @@ fa_status bwd_pre_impl(const void* o, const float* lse, const void* dO, int B, i
     return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// The backward main stage at d = 64 without a bias runs two CTAs per SM
+// (fa_bwd_main64_kernel).  FA_BWD64X2=0 at build time sends it to the 64-row
+// kernel with one CTA per SM instead, for comparisons.
+#ifndef FA_BWD64X2
+#define FA_BWD64X2 1
+#endif
+
 fa_status bwd_main_impl(const void* q, const void* k, const void* v, const void* dO, void* dk,
                         void* dv, int B, int H, int N, int d, int causal, float scale,
                         void* workspace, size_t workspace_bytes, void* stream,
@@ -531,7 +543,12 @@ fa_status bwd_main_impl(const void* q, const void* k, const void* v, const void*
 #define FA_BWD_MAIN(DD, CC, BB)                                                            \
     fa::launch_bwd_main<DD, CC, BB>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv, macc, err, s, \
                                     0, bias, dbias, H, bias_batch, bias_heads, causal == 2)
-    if (bias) {
+    if (FA_BWD64X2 && d == 64 && !bias) {
+        e = causal ? fa::launch_bwd_main64<true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                 macc, err, s, 0, causal == 2)
+                   : fa::launch_bwd_main64<false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                  macc, err, s, 0, 0);
+    } else if (bias) {
         if (d == 64)
             e = causal ? FA_BWD_MAIN(64, true, true) : FA_BWD_MAIN(64, false, true);
         else
@@ -594,7 +611,12 @@ fa_status bwd_accum_impl(const void* q, const void* k, const void* v, const void
 #define FA_BWD_ACC(DD, CC)                                                                  \
     fa::launch_bwd_main<DD, CC>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv, macc, err, s, 1, \
                                 nullptr, nullptr, 1, 0, 0, strict)
-    if (d == 64)
+    if (FA_BWD64X2 && d == 64)
+        e = causal ? fa::launch_bwd_main64<true>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                 macc, err, s, 1, strict)
+                   : fa::launch_bwd_main64<false>(ibh, N, scale, ws, mq, mk, mv, mdo, mdk, mdv,
+                                                  macc, err, s, 1, 0);
+    else if (d == 64)
         e = causal ? FA_BWD_ACC(64, true) : FA_BWD_ACC(64, false);
     else
         e = causal ? FA_BWD_ACC(128, true) : FA_BWD_ACC(128, false);
