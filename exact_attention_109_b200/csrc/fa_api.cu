@@ -15,6 +15,7 @@
 #include "fa_bwd_kernels.cuh"
 #include "fa_decode_kernel.cuh"
 #include "fa_fwd1_kernel.cuh"
+#include "fa_fwd64_kernel.cuh"
 #include "fa_fwd_kernel.cuh"
 #include "fa_merge_kernels.cuh"
 
@@ -144,6 +145,10 @@ fa_status device_setup(int* dev_out, unsigned int** err_out) {
                              fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
         ok &= prepare_kernel(fa::fa_bwd_main_kernel<128, true>, fa::BwdTraits<128>::SMEM_BYTES,
                              fa::BwdTraits<128>::NUM_THREADS, fa::BwdTraits<128>::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd64_kernel<false>, fa::Fwd64Traits::SMEM_BYTES,
+                             fa::Fwd64Traits::NUM_THREADS, fa::Fwd64Traits::REG_BUDGET);
+        ok &= prepare_kernel(fa::fa_fwd64_kernel<true>, fa::Fwd64Traits::SMEM_BYTES,
+                             fa::Fwd64Traits::NUM_THREADS, fa::Fwd64Traits::REG_BUDGET);
         ok &= prepare_kernel(fa::fa_bwd_main64_kernel<false>, fa::Bwd64Traits::SMEM_BYTES,
                              fa::Bwd64Traits::NUM_THREADS, fa::Bwd64Traits::REG_BUDGET);
         ok &= prepare_kernel(fa::fa_bwd_main64_kernel<true>, fa::Bwd64Traits::SMEM_BYTES,
@@ -248,14 +253,18 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
     return cudaGetLastError();
 }
 
-// Short sequences run the forward with one query tile at a time per CTA,
-// two persistent CTAs per SM (fa_fwd1_kernel), which hides the fixed cost
-// around each tile; longer ones use fa_fwd_kernel's two tiles per CTA, which
-// share every K/V block between two tiles.  Measured crossover on a B200
-// (16k tokens per batch, forward TFLOP/s): the one-tile kernel wins up to
-// N = 512 at both head dims (+16-25% d = 64, +9% d = 128) and at N = 1024 for
-// causal d = 64 (+10%); from N = 1024 on it loses up to 19% at d = 128.
-// FA_FWD1_MAX_N overrides the threshold (0: never) for experiments.
+// Forward kernel choice, from same-box measurements (16k tokens per batch,
+// forward TFLOP/s):
+//  * d = 128, N <= 512: one query tile at a time per CTA, two persistent
+//    CTAs per SM (fa_fwd1_kernel), which hides the fixed cost around each
+//    tile (+9% over fa_fwd_kernel); from N = 1024 on it loses up to 19%.
+//  * d = 64, N <= 2048: two tiles per CTA with 64-key blocks and two CTAs
+//    per SM (fa_fwd64_kernel): +24% at N = 512, +10% at N = 1024, +1-5% at
+//    N = 2048 over fa_fwd_kernel, and level with or ahead of the one-tile
+//    kernel; from N = 4096 on it loses 0-7%.
+//  * otherwise fa_fwd_kernel: two tiles per CTA sharing every 128-key block.
+// FA_FWD1_MAX_N overrides the one-tile threshold at both head dims (0:
+// never) for experiments.
 #ifndef FA_FWD1_MAX_N
 #define FA_FWD1_MAX_N -1
 #endif
@@ -266,9 +275,9 @@ cudaError_t launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUten
 #define FA_FWD1_CTAS_PER_SM 2
 #endif
 
-bool use_fwd1(int N, int d, int causal) {
+bool use_fwd1(int N, int d) {
     if (FA_FWD1_MAX_N >= 0) return N <= FA_FWD1_MAX_N;
-    return N <= 512 || (d == 64 && causal && N <= 1024);
+    return d == 128 && N <= 512;
 }
 
 template <int D, bool CAUSAL>
@@ -283,6 +292,25 @@ cudaError_t launch_fwd1(const CUtensorMap& mq, const CUtensorMap& mk, const CUte
     const long long grid = std::min(tiles, cap);
     fa::fa_fwd1_kernel<D, CAUSAL><<<static_cast<unsigned>(grid), T::NUM_THREADS, T::SMEM_BYTES,
                                     stream>>>(mq, mk, mv, mo, prm);
+    return cudaGetLastError();
+}
+
+// FA_FWD64X2=0 at build time leaves d = 64 to fa_fwd_kernel (and the
+// one-tile kernel under FA_FWD1_MAX_N), for comparisons.
+#ifndef FA_FWD64X2
+#define FA_FWD64X2 1
+#endif
+
+bool use_fwd64(int N, int d) { return FA_FWD64X2 && FA_FWD1_MAX_N < 0 && d == 64 && N <= 2048; }
+
+template <bool CAUSAL>
+cudaError_t launch_fwd64(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& mo, const fa::FwdParams& prm, long long bh,
+                         cudaStream_t stream) {
+    using T = fa::Fwd64Traits;
+    const long long grid = bh * prm.n_qpairs;
+    fa::fa_fwd64_kernel<CAUSAL><<<static_cast<unsigned>(grid), T::NUM_THREADS, T::SMEM_BYTES,
+                                  stream>>>(mq, mk, mv, mo, prm);
     return cudaGetLastError();
 }
 
@@ -340,7 +368,15 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     prm.strict = causal == 2;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (use_fwd1(N, d, causal)) {
+    if (use_fwd64(N, d)) {
+        CUtensorMap mk64, mv64;  // 64-key boxes
+        if (!encode_bf16(&mk64, k, d, N, bh, 64) || !encode_bf16(&mv64, v, d, N, bh, 64))
+            return FA_ERR_CUDA;
+        e = causal ? launch_fwd64<true>(mq, mk64, mv64, mo, prm, bh, s)
+                   : launch_fwd64<false>(mq, mk64, mv64, mo, prm, bh, s);
+        return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+    }
+    if (use_fwd1(N, d)) {
         if (d == 64)
             e = causal ? launch_fwd1<64, true>(mq, mk, mv, mo, prm, bh, g_dev[dev].sm_count, s)
                        : launch_fwd1<64, false>(mq, mk, mv, mo, prm, bh, g_dev[dev].sm_count, s);
