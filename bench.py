@@ -42,6 +42,8 @@ WORKLOADS = {
                                             dist="normal", seed=2),
     "fwd_bwd_sweep_N8192_d64_causal": dict(B=2, H=32, N=8192, d=64, causal=True,
                                            dist="normal", seed=2),
+    "fwd_bwd_sweep_N2048_d64_causal": dict(B=8, H=32, N=2048, d=64, causal=True,
+                                           dist="normal", seed=2),
     "fwd_bwd_sweep_N8192_d128_noncausal": dict(B=2, H=16, N=8192, d=128, causal=False,
                                                dist="normal", seed=2),
     "gpt_layer_a_B8_N2048_H16_d128": dict(B=8, H=16, N=2048, d=128, causal=True,
@@ -120,10 +122,28 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "fa_fwd_kernel": "fa_fwd_kernel.cuh",
-    "fa_bwd_main_kernel": "fa_bwd_kernels.cuh",
-    "fa_decode_kernel": "fa_decode_kernel.cuh",
+    "fa_fwd_kernel": ("fa_fwd_kernel.cuh",),
+    "fa_fwd1_kernel": ("fa_fwd1_kernel.cuh", "fa_fwd_kernel.cuh"),
+    "fa_fwd64_kernel": ("fa_fwd64_kernel.cuh", "fa_fwd_kernel.cuh"),
+    "fa_bwd_main_kernel": ("fa_bwd_kernels.cuh",),
+    "fa_bwd_main64_kernel": ("fa_bwd64_kernel.cuh", "fa_bwd_kernels.cuh"),
+    "fa_decode_kernel": ("fa_decode_kernel.cuh",),
 }
+
+
+def fwd_kernel_name(N: int, d: int) -> str:
+    """The forward kernel fa_fwd launches for this shape (the shape rule in
+    csrc/fa_api.cu, use_fwd64 and use_fwd1)."""
+    if d == 64 and N <= 2048:
+        return "fa_fwd64_kernel"
+    if d == 128 and N <= 512:
+        return "fa_fwd1_kernel"
+    return "fa_fwd_kernel"
+
+
+def bwd_main_kernel_name(d: int) -> str:
+    """The backward main-stage kernel fa_bwd_main launches (no bias)."""
+    return "fa_bwd_main64_kernel" if d == 64 else "fa_bwd_main_kernel"
 
 
 # Files besides the kernel's own that decide what it does: the PTX helpers
@@ -134,7 +154,7 @@ SHARED_SOURCES = ("sm100_ptx.cuh", "fa_api.cu")
 def kernel_sources_hash(kernel: str) -> str:
     """Hash of the kernel's own source file and of the shared sources above."""
     h = hashlib.sha256()
-    for name in (KERNEL_SOURCES[kernel],) + SHARED_SOURCES:
+    for name in KERNEL_SOURCES[kernel] + SHARED_SOURCES:
         with open(os.path.join(ROOT, "exact_attention_109_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -402,8 +422,8 @@ def gpu_arm(args, w, wname):
     def stage_conv():
         return fa.fa_bwd_dq_convert(P["dq"], B, H, N, d, scale, P["ws"], ws_bytes, s)
 
-    stages = [("fa_fwd_kernel", stage_fwd), ("fa_bwd_pre_kernel", stage_pre),
-              ("fa_bwd_main_kernel", stage_main), ("fa_bwd_dq_convert_kernel", stage_conv)]
+    stages = [(fwd_kernel_name(N, d), stage_fwd), ("fa_bwd_pre_kernel", stage_pre),
+              (bwd_main_kernel_name(d), stage_main), ("fa_bwd_dq_convert_kernel", stage_conv)]
 
     def step(events=None):
         for i, (_, fn) in enumerate(stages):
@@ -525,8 +545,8 @@ def gpu_arm(args, w, wname):
     bh = B * H
     n_pad = (N + 127) // 128 * 128
     algo = {
-        "fa_fwd_kernel": ("tensor", fwd_flops(w)),
-        "fa_bwd_main_kernel": ("tensor", 2.5 * fwd_flops(w)),
+        fwd_kernel_name(N, d): ("tensor", fwd_flops(w)),
+        bwd_main_kernel_name(d): ("tensor", 2.5 * fwd_flops(w)),
         "fa_bwd_pre_kernel": ("hbm", 2 * bh * N * d * 2 + bh * N * 4 + 2 * bh * n_pad * 4
                               + bh * n_pad * d * 4),
         "fa_bwd_dq_convert_kernel": ("hbm", bh * N * d * 4 + bh * N * d * 2),
