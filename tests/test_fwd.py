@@ -7,8 +7,8 @@ import torch
 
 import exact_attention_109_b200 as fa
 from exact_attention_109_b200.inputs import default_scale
-from parity_util import (check_forward_full, check_forward_sampled, gpu_inputs,
-                         run_forward)
+from parity_util import (check_forward_full, check_forward_sampled, check_full, gpu_inputs,
+                         run_backward, run_forward)
 
 pytestmark = pytest.mark.gpu
 
@@ -28,6 +28,19 @@ def test_ragged_lengths(N, causal, d):
     host, dev = gpu_inputs(2, 3, N, d, seed=N + 17 * d + int(causal))
     o, lse = run_forward(dev, causal, default_scale(d))
     check_forward_full(host, o, lse, causal, default_scale(d))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N,d", [(512, 128), (513, 128), (2048, 64), (2049, 64)])
+def test_kernel_crossovers(N, d, causal):
+    """fa_fwd picks its kernel by shape: the lengths on either side of each
+    switch (d = 128: one-tile up to N = 512; d = 64: 64-key blocks up to
+    N = 2048), whole tensors, forward and backward."""
+    host, dev = gpu_inputs(1, 2, N, d, seed=N + 3 * d + int(causal), with_dout=True)
+    scale = default_scale(d)
+    o, lse = run_forward(dev, causal, scale)
+    dq, dk, dv = run_backward(dev, o, lse, causal, scale)
+    check_full(host, o, lse, dq, dk, dv, causal, scale)
 
 
 @pytest.mark.parametrize("d", [64, 128])
