@@ -90,8 +90,8 @@ struct FwdTraits {
     static constexpr int LOAD_WARP = 9;
     static constexpr int BIAS_WARP = 10;
     // Register split: softmax warpgroups grow, the MMA/TMA warpgroup shrinks.
-    static constexpr uint32_t REG_SOFTMAX = 208;
-    static constexpr uint32_t REG_CONTROL = 88;
+    static constexpr uint32_t REG_SOFTMAX = 200;
+    static constexpr uint32_t REG_CONTROL = 104;
     static constexpr int REG_BUDGET = 128 * (2 * REG_SOFTMAX + REG_CONTROL);
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC_S = QK8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, 0, 0);
@@ -389,24 +389,31 @@ __global__ void __launch_bounds__(384, 1)
         __syncwarp();
       } else if (warp == T::MMA_WARP) {
         // ------------------------------------------------ MMA issuer
+        // This one thread's instruction stream paces the kernel: it shares
+        // its SM sub-partition with two busy softmax warps, and a probe that
+        // added 32 dependent integer instructions per key block cost 8-12%
+        // of the forward's rate.  So what does not change from block to
+        // block is computed once (operand descriptors, barrier addresses)
+        // and the ring position advances by adds.
         if (lane == 0) {
             const uint32_t q_base = smem_u32(smem + T::Q_OFF);
             const uint32_t kv_base = smem_u32(smem + T::KV_OFF);
-            auto slot_addr = [&](int idx) {
-                return kv_base + static_cast<uint32_t>((idx % T::NSLOT) * T::TILE_BYTES);
-            };
-            auto slot_par = [&](int idx) { return static_cast<uint32_t>((idx / T::NSLOT) & 1); };
+            const uint64_t dq[2] = {sdesc_sw128(q_base, 16, 1024),
+                                    sdesc_sw128(q_base + T::QK_TILE_BYTES, 16, 1024)};
+            const uint64_t dk_base = sdesc_sw128(kv_base, 16, 1024);             // K in slot 0
+            const uint64_t dv_base = sdesc_sw128(kv_base, T::CHUNK_BYTES, 1024);  // V in slot 0
+            const uint32_t full_a = smem_u32(full), empty_a = smem_u32(empty);
+            const uint32_t sfull_a = smem_u32(s_full), pready_a = smem_u32(p_ready);
+            const uint32_t phalf_a = smem_u32(p_half), ofinal_a = smem_u32(o_final);
             // S_t = Q_t K^T : M=128, N=128, K=D, both operands K-major;
             // each MMA consumes 32 bytes of every row (16 bf16 or 32 e4m3).
-            // Descriptors: one base per tile, K steps add byte offsets.
-            auto mma_s = [&](int t, uint32_t k_addr) {
-                const uint64_t dq0 = sdesc_sw128(q_base + t * T::QK_TILE_BYTES, 16, 1024);
-                const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
+            // dk: the descriptor of the K slot; K steps add byte offsets.
+            auto mma_s = [&](int t, uint64_t dk) {
 #pragma unroll
                 for (int k = 0; k < T::S_KSTEPS; ++k) {
                     const uint32_t off = (k >> 2) * T::CHUNK_BYTES + (k & 3) * 32;
-                    const uint64_t a = sdesc_add(dq0, off);
-                    const uint64_t b = sdesc_add(dk0, off);
+                    const uint64_t a = sdesc_add(dq[t], off);
+                    const uint64_t b = sdesc_add(dk, off);
                     if constexpr (QK8)
                         umma_ss_f8(tmem + 128u * t, a, b, T::IDESC_S, k > 0 ? 1u : 0u);
                     else if (k == 0)
@@ -416,13 +423,12 @@ __global__ void __launch_bounds__(384, 1)
                 }
             };
             // O_t += P_t V : M=128, N=D, K=128; P from TMEM, V MN-major.
-            // K steps [k0, k1) of O_t += P_t V (16 keys each).
-            auto mma_pv = [&](int t, uint32_t v_addr, bool accumulate, int k0, int k1) {
-                const uint64_t dv0 = sdesc_sw128(v_addr, T::CHUNK_BYTES, 1024);
+            // K steps [k0, k1) of O_t += P_t V (16 keys each); dv: the V slot.
+            auto mma_pv = [&](int t, uint64_t dv, bool accumulate, int k0, int k1) {
 #pragma unroll
                 for (int k = k0; k < k1; ++k) {
                     const uint32_t a = tmem + 128u * t + 8u * k;  // 32 bytes of P per row
-                    const uint64_t b = sdesc_add(dv0, k * T::PV_KSTEP_BYTES);
+                    const uint64_t b = sdesc_add(dv, k * T::PV_KSTEP_BYTES);
                     const uint32_t acc = (k > 0 || accumulate) ? 1u : 0u;
                     if constexpr (PV8)
                         umma_ts_f8(tmem + 256u + D * t, a, b, T::IDESC_PV, acc);
@@ -434,68 +440,84 @@ __global__ void __launch_bounds__(384, 1)
             };
             // PV of tile t for the block whose P has phase `par`: in two
             // 64-key halves when the softmax signals them separately.
-            auto pv_tile = [&](int t, uint32_t v_addr, bool acc, uint32_t par) -> bool {
+            auto pv_tile = [&](int t, uint64_t dv, bool acc, uint32_t par) -> bool {
                 if constexpr (T::PSPLIT) {
-                    if (!mbar_wait(&p_half[t], par, st)) return false;
+                    if (!mbar_wait_s(phalf_a + 8u * t, par, st)) return false;
                     tc_fence_after();
-                    mma_pv(t, v_addr, acc, 0, T::PV_KSTEPS / 2);
-                    if (!mbar_wait(&p_ready[t], par, st)) return false;
+                    mma_pv(t, dv, acc, 0, T::PV_KSTEPS / 2);
+                    if (!mbar_wait_s(pready_a + 8u * t, par, st)) return false;
                     tc_fence_after();
-                    mma_pv(t, v_addr, true, T::PV_KSTEPS / 2, T::PV_KSTEPS);
+                    mma_pv(t, dv, true, T::PV_KSTEPS / 2, T::PV_KSTEPS);
                 } else {
-                    if (!mbar_wait(&p_ready[t], par, st)) return false;
+                    if (!mbar_wait_s(pready_a + 8u * t, par, st)) return false;
                     tc_fence_after();
-                    mma_pv(t, v_addr, acc, 0, T::PV_KSTEPS);
+                    mma_pv(t, dv, acc, 0, T::PV_KSTEPS);
                 }
                 return true;
             };
-            // Tile 0 takes part in iterations [off0, off0 + n0); its own block
-            // count (for its barrier phases) is i - off0.
-            auto act0 = [&](int i) { return i >= off0 && i - off0 < n0; };
-            bool ok = mbar_wait(bar_q, 0, st) && mbar_wait(&full[0], 0, st);
+            // Tile 0 takes part in iterations [off0, n1) (off0 + n0 = n1);
+            // its own block count (for its barrier phases) is i - off0.
+            auto act0 = [&](int i) { return i >= off0; };
+            bool ok = mbar_wait(bar_q, 0, st) && mbar_wait_s(full_a, 0, st);
             if (ok) {
                 tc_fence_after();
                 if (act0(0)) {
-                    mma_s(0, slot_addr(0));
-                    umma_commit(&s_full[0]);
+                    mma_s(0, dk_base);
+                    umma_commit_s(sfull_a);
                 }
-                mma_s(1, slot_addr(0));
-                umma_commit(&s_full[1]);
-                umma_commit(&empty[0]);
+                mma_s(1, dk_base);
+                umma_commit_s(sfull_a + 8u);
+                umma_commit_s(empty_a);
             }
+            // Ring slot and phase parity of K_j (position 2j); V_{j-1} sits
+            // one position before it.
+            uint32_t ks = 2u % T::NSLOT, kp = (2u / T::NSLOT) & 1u;
             for (int j = 1; j < n1 && ok; ++j) {
-                const int ik = 2 * j, iv = 2 * j - 1;  // K of iteration j, V of j-1
-                ok = mbar_wait(&full[ik % T::NSLOT], slot_par(ik), st) &&
-                     mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st);
+                const uint32_t vs = ks ? ks - 1u : T::NSLOT - 1u;
+                const uint32_t vp = ks ? kp : kp ^ 1u;
+                ok = mbar_wait_s(full_a + 8u * ks, kp, st) && mbar_wait_s(full_a + 8u * vs, vp, st);
                 if (!ok) break;
                 tc_fence_after();
+                const uint64_t dk = sdesc_add(dk_base, ks * T::TILE_BYTES);
+                const uint64_t dv = sdesc_add(dv_base, vs * T::TILE_BYTES);
                 if (act0(j - 1)) {
-                    const int l0 = j - 1 - off0;
-                    if (!(ok = pv_tile(0, slot_addr(iv), l0 > 0, l0 & 1))) break;
-                    if (l0 == n0 - 1) umma_commit(&o_final[0]);
+                    const int l0 = j - 1 - off0;  // never tile 0's last block (that is j = n1)
+                    if (!(ok = pv_tile(0, dv, l0 > 0, l0 & 1))) break;
                 }
                 if (act0(j)) {
-                    mma_s(0, slot_addr(ik));
-                    umma_commit(&s_full[0]);
+                    mma_s(0, dk);
+                    umma_commit_s(sfull_a);
                 }
-                if (!(ok = pv_tile(1, slot_addr(iv), j - 1 > 0, (j - 1) & 1))) break;
-                umma_commit(&empty[iv % T::NSLOT]);
-                mma_s(1, slot_addr(ik));
-                umma_commit(&s_full[1]);
-                umma_commit(&empty[ik % T::NSLOT]);
+                if (!(ok = pv_tile(1, dv, j - 1 > 0, (j - 1) & 1))) break;
+                umma_commit_s(empty_a + 8u * vs);
+                mma_s(1, dk);
+                umma_commit_s(sfull_a + 8u);
+                umma_commit_s(empty_a + 8u * ks);
+                ks += 2u;
+                if (ks >= T::NSLOT) {
+                    ks -= T::NSLOT;
+                    kp ^= 1u;
+                }
             }
-            if (ok) {
-                const int jl = n1 - 1, iv = 2 * n1 - 1;
-                ok = mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st);
+            if (ok) {  // V of the last block, one position before K_{n1}'s
+                const int jl = n1 - 1;
+                const uint32_t vs = ks ? ks - 1u : T::NSLOT - 1u;
+                const uint32_t vp = ks ? kp : kp ^ 1u;
+                const uint64_t dv = sdesc_add(dv_base, vs * T::TILE_BYTES);
+                ok = mbar_wait_s(full_a + 8u * vs, vp, st);
                 if (ok && act0(jl)) {
+                    tc_fence_after();
                     const int l0 = jl - off0;
-                    ok = pv_tile(0, slot_addr(iv), l0 > 0, l0 & 1);
-                    if (ok) umma_commit(&o_final[0]);
+                    ok = pv_tile(0, dv, l0 > 0, l0 & 1);
+                    if (ok) umma_commit_s(ofinal_a);
                 }
-                if (ok) ok = pv_tile(1, slot_addr(iv), jl > 0, jl & 1);
                 if (ok) {
-                    umma_commit(&o_final[1]);
-                    umma_commit(&empty[iv % T::NSLOT]);
+                    tc_fence_after();
+                    ok = pv_tile(1, dv, jl > 0, jl & 1);
+                }
+                if (ok) {
+                    umma_commit_s(ofinal_a + 8u);
+                    umma_commit_s(empty_a + 8u * vs);
                 }
             }
             // No MMA may still be running when TMEM is released.

@@ -95,6 +95,37 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
     }
 }
 
+// mbar_wait on a barrier given by its shared-window address, for the
+// MMA-issuing threads: their instruction streams pace the kernels, so their
+// hot loops keep barrier addresses in registers and skip the conversion.
+__device__ __forceinline__ bool mbar_try_wait_s(uint32_t addr, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(ok)
+        : "r"(addr), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ bool mbar_wait_s(uint32_t addr, uint32_t parity, const AbortState& st,
+                                            unsigned long long limit_ns = kWaitLimitNs) {
+    if (mbar_try_wait_s(addr, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait_s(addr, parity)) return true;
+        if ((it & 31u) == 0u) {
+            if (*st.flag) return false;
+            if (globaltimer_ns() - t0 > limit_ns) {
+                raise_abort(st);
+                return false;
+            }
+        }
+    }
+}
+
 // Same, but without the abort flag (used for clean-up waits after an abort).
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
     const unsigned long long t0 = globaltimer_ns();
@@ -287,6 +318,13 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_u32(bar))
+        : "memory");
+}
+
+// umma_commit on a barrier given by its shared-window address.
+__device__ __forceinline__ void umma_commit_s(uint32_t addr) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(addr)
         : "memory");
 }
 
