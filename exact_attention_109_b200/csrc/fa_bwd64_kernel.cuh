@@ -186,9 +186,20 @@ __global__ void __launch_bounds__(256, 2) fa_bwd_main64_kernel(
         __syncwarp();
       } else if (warp == T::MMA_WARP) {
         // ------------------------------------------------ MMA issuer
+        // This thread paces the kernel, so the stage descriptors and barrier
+        // addresses are built once and the stage ring advances by adds.
         if (lane == 0) {
             const uint32_t k_base = smem_u32(smem + T::K_OFF);
             const uint32_t st_base = smem_u32(smem + T::ST_OFF);
+            // Stage 0's Q and dO, K-major (S^T, dP^T) and MN-major (dV, dK);
+            // stage s adds s * STAGE_BYTES.
+            const uint64_t sq_k = sdesc_sw128(st_base, 16, 1024);
+            const uint64_t sdo_k = sdesc_sw128(st_base + T::Q_TILE, 16, 1024);
+            const uint64_t sq_mn = sdesc_sw128(st_base, T::Q_TILE, 1024);
+            const uint64_t sdo_mn = sdesc_sw128(st_base + T::Q_TILE, T::Q_TILE, 1024);
+            const uint32_t sfull_a = smem_u32(stage_full), sempty_a = smem_u32(stage_empty);
+            const uint32_t sdpf_a = smem_u32(sdp_full), pds_a = smem_u32(pds_ready);
+            const uint32_t dqf_a = smem_u32(dq_full), dqd_a = smem_u32(dq_drained);
             const uint64_t dk0 = sdesc_sw128(k_base, 16, 1024);
             const uint64_t dv0 = sdesc_sw128(smem_u32(smem + T::V_OFF), 16, 1024);
             // K^T as the A operand of dQ^T, MN-major: M = 128 rows of which
@@ -198,10 +209,9 @@ __global__ void __launch_bounds__(256, 2) fa_bwd_main64_kernel(
             const uint64_t dds0 = sdesc_sw128(smem_u32(smem + T::DS_OFF), T::DS_TILE, 1024);
             // S^T = K Q^T into [0, 64) and dP^T = V dO^T into [64, 128):
             // M = 128 keys, N = 64 queries, K = 64 head dims.
-            auto mma_sdp = [&](int k) {
-                const uint32_t sq = st_base + (k % T::NSTAGE) * T::STAGE_BYTES;
-                const uint64_t dq0 = sdesc_sw128(sq, 16, 1024);
-                const uint64_t ddo0 = sdesc_sw128(sq + T::Q_TILE, 16, 1024);
+            auto mma_sdp = [&](uint32_t soff) {  // soff: the stage's byte offset
+                const uint64_t dq0 = sdesc_add(sq_k, soff);
+                const uint64_t ddo0 = sdesc_add(sdo_k, soff);
                 umma_ss_c<false>(tmem + T::S_COL, dk0, dq0, T::IDESC_SDP);
 #pragma unroll
                 for (int kk = 1; kk < D / 16; ++kk)
@@ -216,11 +226,10 @@ __global__ void __launch_bounds__(256, 2) fa_bwd_main64_kernel(
             // dV += P^T dO and dK += dS^T Q: M = 128 keys, N = 64 head dims,
             // K = 64 queries; A (P^T at [0, 32), dS^T at [64, 96)) from TMEM,
             // B (dO or Q) MN-major from the stage.
-            auto mma_dkdv = [&](int k) {
-                const uint32_t sq = st_base + (k % T::NSTAGE) * T::STAGE_BYTES;
-                const uint64_t bq0 = sdesc_sw128(sq, T::Q_TILE, 1024);
-                const uint64_t bdo0 = sdesc_sw128(sq + T::Q_TILE, T::Q_TILE, 1024);
-                const uint32_t acc = k > 0 ? 1u : 0u;  // the first block overwrites
+            auto mma_dkdv = [&](uint32_t soff, bool first) {
+                const uint64_t bq0 = sdesc_add(sq_mn, soff);
+                const uint64_t bdo0 = sdesc_add(sdo_mn, soff);
+                const uint32_t acc = first ? 0u : 1u;  // the first block overwrites
                 umma_ts(tmem + T::DV_COL, tmem + T::S_COL, bdo0, T::IDESC_ACC, acc);
                 umma_ts(tmem + T::DK_COL, tmem + T::DP_COL, bq0, T::IDESC_ACC, acc);
 #pragma unroll
@@ -240,33 +249,39 @@ __global__ void __launch_bounds__(256, 2) fa_bwd_main64_kernel(
                     umma_ss_c<true>(tmem + T::DP_COL, sdesc_add(dkt0, kk * 2048),
                                     sdesc_add(dds0, kk * 2048), T::IDESC_DQ);
             };
-            bool ok = mbar_wait(bar_kv, 0, st) && mbar_wait(&stage_full[0], 0, st);
+            bool ok = mbar_wait(bar_kv, 0, st) && mbar_wait_s(sfull_a, 0, st);
             if (ok) {
                 tc_fence_after();
                 mma_sdp(0);
-                umma_commit(sdp_full);
+                umma_commit_s(sdpf_a);
             }
+            // Stage slot of block k (s0) and of block k+1 (s1, with its
+            // phase parity p1), advanced by one slot per block.
+            uint32_t s0 = 0, s1 = 1u % T::NSTAGE, p1 = (1u / T::NSTAGE) & 1u;
             for (int k = 0; k < n && ok; ++k) {
-                if (!(ok = mbar_wait(pds_ready, k & 1, st))) break;
+                if (!(ok = mbar_wait_s(pds_a, k & 1, st))) break;
                 tc_fence_after();
-                mma_dkdv(k);
+                mma_dkdv(s0 * T::STAGE_BYTES, k == 0);
                 // dQ^T takes the dP^T columns after dK above has read dS^T
                 // from them (MMAs from one thread run in order).
                 mma_dq();
-                umma_commit(dq_full);
-                umma_commit(&stage_empty[k % T::NSTAGE]);
+                umma_commit_s(dqf_a);
+                umma_commit_s(sempty_a + 8u * s0);
                 if (k + 1 < n) {
                     // S^T(k+1) overwrites P^T(k) after dV(k) has read it (in
                     // order); dP^T(k+1) waits for the drain to have read
                     // dQ^T(k).  Their commit also covers dQ^T(k), the last
                     // reader of the dS^T tile that block k+1 rewrites.
-                    if (!(ok = mbar_wait(&stage_full[(k + 1) % T::NSTAGE],
-                                         ((k + 1) / T::NSTAGE) & 1, st)))
-                        break;
-                    if (!(ok = mbar_wait(dq_drained, k & 1, st))) break;
+                    if (!(ok = mbar_wait_s(sfull_a + 8u * s1, p1, st))) break;
+                    if (!(ok = mbar_wait_s(dqd_a, k & 1, st))) break;
                     tc_fence_after();
-                    mma_sdp(k + 1);
-                    umma_commit(sdp_full);
+                    mma_sdp(s1 * T::STAGE_BYTES);
+                    umma_commit_s(sdpf_a);
+                }
+                if (++s0 == T::NSTAGE) s0 = 0;
+                if (++s1 == T::NSTAGE) {
+                    s1 = 0;
+                    p1 ^= 1u;
                 }
             }
             if (ok) umma_commit(kv_done);

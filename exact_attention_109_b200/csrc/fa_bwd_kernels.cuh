@@ -331,6 +331,11 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
         __syncwarp();
       } else if (warp == T::MMA_WARP) {
         // ------------------------------------------------ MMA issuer
+        // This one thread paces the kernel (the P/dS results wait for it),
+        // so its hot loop does as little else as possible: the operand
+        // descriptors of stage 0, the dS^T buffers and the fixed tiles are
+        // built once, barrier addresses stay in registers, and the stage
+        // ring advances by adds (no % or / by the stage count).
         if (lane == 0) {
             const uint32_t k_base = smem_u32(smem + T::K_OFF);
             const uint32_t v_base = smem_u32(smem + T::V_OFF);
@@ -341,10 +346,20 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
             const uint64_t dk0 = sdesc_sw128(k_base, 16, 1024);
             const uint64_t dv0 = sdesc_sw128(v_base, 16, 1024);
             const uint64_t dkt0 = sdesc_sw128(k_base, T::KV_CHUNK, 1024);
-            auto mma_sdp = [&](int k, int b) {
-                const uint32_t sq = st_base + (k % T::NSTAGE) * T::STAGE_BYTES;
-                const uint64_t dq0 = sdesc_sw128(sq, 16, 1024);
-                const uint64_t ddo0 = sdesc_sw128(sq + T::Q_TILE, 16, 1024);
+            // Stage 0's Q and dO, K-major (S^T, dP^T) and MN-major (dV, dK);
+            // stage s adds s * STAGE_BYTES.
+            const uint64_t sq_k = sdesc_sw128(st_base, 16, 1024);
+            const uint64_t sdo_k = sdesc_sw128(st_base + T::Q_TILE, 16, 1024);
+            const uint64_t sq_mn = sdesc_sw128(st_base, T::Q_CHUNK, 1024);
+            const uint64_t sdo_mn = sdesc_sw128(st_base + T::Q_TILE, T::Q_CHUNK, 1024);
+            const uint64_t dds_b0 = sdesc_sw128(ds_base, T::DS_TILE, 1024);  // dS^T buffer 0
+            const uint32_t sfull_a = smem_u32(stage_full), sempty_a = smem_u32(stage_empty);
+            const uint32_t sdpf_a = smem_u32(sdp_full), sdpl_a = smem_u32(sdp_loaded);
+            const uint32_t pds_a = smem_u32(pds_ready), dqf_a = smem_u32(dq_full);
+            const uint32_t dqd_a = smem_u32(dq_drained);
+            auto mma_sdp = [&](uint32_t soff, int b) {  // soff: the stage's byte offset
+                const uint64_t dq0 = sdesc_add(sq_k, soff);
+                const uint64_t ddo0 = sdesc_add(sdo_k, soff);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint32_t offk = (kk >> 2) * T::KV_CHUNK + (kk & 3) * 32;
@@ -368,16 +383,16 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
             };
             // dV += P^T dO and dK += dS^T Q: M=128 keys, N=D, K=64 queries;
             // A (P^T or dS^T) from TMEM, B (dO or Q) MN-major from the stage.
-            auto mma_dkdv = [&](int k, int b) {
-                const uint32_t sq = st_base + (k % T::NSTAGE) * T::STAGE_BYTES;
-                const uint64_t bq0 = sdesc_sw128(sq, T::Q_CHUNK, 1024);
-                const uint64_t bdo0 = sdesc_sw128(sq + T::Q_TILE, T::Q_CHUNK, 1024);
+            auto mma_dkdv = [&](uint32_t soff, bool first, int b) {
+                const uint64_t bq0 = sdesc_add(sq_mn, soff);
+                const uint64_t bdo0 = sdesc_add(sdo_mn, soff);
 #pragma unroll
                 for (int kk = 0; kk < T::BM / 16; ++kk) {
                     const uint32_t a_col = 128u * b + 32u * (kk >> 1) + 8u * (kk & 1);
                     if (kk == 0) {  // the first query block overwrites, later ones accumulate
-                        umma_ts(tmem + T::DV_COL, tmem + a_col, bdo0, T::IDESC_ACC, k > 0);
-                        umma_ts(tmem + T::DK_COL, tmem + a_col + 16u, bq0, T::IDESC_ACC, k > 0);
+                        umma_ts(tmem + T::DV_COL, tmem + a_col, bdo0, T::IDESC_ACC, first ? 0u : 1u);
+                        umma_ts(tmem + T::DK_COL, tmem + a_col + 16u, bq0, T::IDESC_ACC,
+                                first ? 0u : 1u);
                     } else {
                         umma_ts_c<true>(tmem + T::DV_COL, tmem + a_col, sdesc_add(bdo0, kk * 2048),
                                         T::IDESC_ACC);
@@ -388,8 +403,8 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
             };
             // dQ^T = K^T dS^T: M=128 (head dim; rows >= D unused), N=64
             // queries, K=128 keys; both operands MN-major in shared memory.
-            auto mma_dq = [&](int k, int b1) {
-                const uint64_t dds0 = sdesc_sw128(ds_base + (k & 1) * T::DS_TILE, T::DS_TILE, 1024);
+            auto mma_dq = [&](int bs, int b1) {  // bs: the dS^T buffer
+                const uint64_t dds0 = sdesc_add(dds_b0, bs * T::DS_TILE);
 #pragma unroll
                 for (int kk = 0; kk < T::BN / 16; ++kk) {
                     if (kk == 0)
@@ -400,37 +415,45 @@ __global__ void __launch_bounds__(512, 1) fa_bwd_main_kernel(
                 }
             };
             bool ok = mbar_wait(bar_kv, 0, st);
-            for (int k = 0; k < 2 && k < n && ok; ++k) {
-                ok = mbar_wait(&stage_full[k % T::NSTAGE], (k / T::NSTAGE) & 1, st);
+            for (int k = 0; k < 2 && k < n && ok; ++k) {  // stages 0 and 1, phase 0
+                ok = mbar_wait_s(sfull_a + 8u * k, 0, st);
                 if (!ok) break;
                 tc_fence_after();
-                mma_sdp(k, k);
-                umma_commit(&sdp_full[k]);
+                mma_sdp(static_cast<uint32_t>(k) * T::STAGE_BYTES, k);
+                umma_commit_s(sdpf_a + 8u * k);
             }
+            // Stage slot of block k (s0) and of block k+2 (s2, with its phase
+            // parity p2), advanced by one slot per block.
+            uint32_t s0 = 0, s2 = 2u % T::NSTAGE, p2 = (2u / T::NSTAGE) & 1u;
             for (int k = 0; k < n && ok; ++k) {
                 const int b = k & 1, b1 = b ^ 1;
-                if (!(ok = mbar_wait(&pds_ready[b], (k >> 1) & 1, st))) break;
+                if (!(ok = mbar_wait_s(pds_a + 8u * b, (k >> 1) & 1, st))) break;
                 tc_fence_after();
-                mma_dkdv(k, b);
+                mma_dkdv(s0 * T::STAGE_BYTES, k == 0, b);
                 if (k + 1 < n)
-                    ok = mbar_wait(&sdp_loaded[b1], ((k + 1) >> 1) & 1, st);
+                    ok = mbar_wait_s(sdpl_a + 8u * b1, ((k + 1) >> 1) & 1, st);
                 else if (k >= 2)
-                    ok = mbar_wait(&dq_drained[b1], ((k - 2) >> 1) & 1, st);
+                    ok = mbar_wait_s(dqd_a + 8u * b1, ((k - 2) >> 1) & 1, st);
                 if (!ok) break;
                 tc_fence_after();
-                mma_dq(k, b1);
-                umma_commit(&dq_full[b1]);
-                umma_commit(&stage_empty[k % T::NSTAGE]);
+                mma_dq(b, b1);
+                umma_commit_s(dqf_a + 8u * b1);
+                umma_commit_s(sempty_a + 8u * s0);
                 if (k + 2 < n) {
-                    ok = mbar_wait(&stage_full[(k + 2) % T::NSTAGE], ((k + 2) / T::NSTAGE) & 1, st);
-                    if (ok && k >= 1) ok = mbar_wait(&dq_drained[b], ((k - 1) >> 1) & 1, st);
+                    ok = mbar_wait_s(sfull_a + 8u * s2, p2, st);
+                    if (ok && k >= 1) ok = mbar_wait_s(dqd_a + 8u * b, ((k - 1) >> 1) & 1, st);
                     if (!ok) break;
                     tc_fence_after();
-                    mma_sdp(k + 2, b);
+                    mma_sdp(s2 * T::STAGE_BYTES, b);
                     // This commit completes only after dQ^T(k) above has read
                     // dS^T buffer k & 1, which block k+2's P/dS warps rewrite
                     // once they see it: keep S/dP(k+2) after dQ^T(k).
-                    umma_commit(&sdp_full[b]);
+                    umma_commit_s(sdpf_a + 8u * b);
+                }
+                if (++s0 == T::NSTAGE) s0 = 0;
+                if (++s2 == T::NSTAGE) {
+                    s2 = 0;
+                    p2 ^= 1u;
                 }
             }
             if (ok) umma_commit(kv_done);

@@ -214,27 +214,30 @@ __global__ void __launch_bounds__(256, 2)
         __syncwarp();
       } else if (warp == T::MMA_WARP) {
         // ------------------------------------------------ MMA issuer
+        // This thread's instruction stream is on the kernel's critical path,
+        // so descriptors and barrier addresses are built once and the ring
+        // position advances by adds (as in fa_fwd_kernel).
         if (lane == 0) {
             const uint32_t q_base = smem_u32(smem + T::Q_OFF);
             const uint32_t kv_base = smem_u32(smem + T::KV_OFF);
-            auto slot_addr = [&](int idx) {
-                return kv_base + static_cast<uint32_t>((idx % T::NSLOT) * T::KV_TILE);
-            };
-            auto slot_par = [&](int idx) { return static_cast<uint32_t>((idx / T::NSLOT) & 1); };
+            const uint64_t dq[2] = {sdesc_sw128(q_base, 16, 1024),
+                                    sdesc_sw128(q_base + T::Q_TILE, 16, 1024)};
+            const uint64_t dk_base = sdesc_sw128(kv_base, 16, 1024);        // K in slot 0
+            const uint64_t dv_base = sdesc_sw128(kv_base, T::KV_TILE, 1024);  // V in slot 0
+            const uint32_t full_a = smem_u32(full), empty_a = smem_u32(empty);
+            const uint32_t sfull_a = smem_u32(s_full), pready_a = smem_u32(p_ready);
+            const uint32_t ofinal_a = smem_u32(o_final);
             // S_t = Q_t K^T: M = 128, N = 64 keys, K = 64 dims, both K-major.
-            auto mma_s = [&](int t, uint32_t k_addr) {
-                const uint64_t dq0 = sdesc_sw128(q_base + t * T::Q_TILE, 16, 1024);
-                const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
-                umma_ss_c<false>(tmem + 64u * t, dq0, dk0, T::IDESC_S);
+            auto mma_s = [&](int t, uint64_t dk0) {
+                umma_ss_c<false>(tmem + 64u * t, dq[t], dk0, T::IDESC_S);
 #pragma unroll
                 for (int k = 1; k < D / 16; ++k)
-                    umma_ss_c<true>(tmem + 64u * t, sdesc_add(dq0, k * 32), sdesc_add(dk0, k * 32),
+                    umma_ss_c<true>(tmem + 64u * t, sdesc_add(dq[t], k * 32), sdesc_add(dk0, k * 32),
                                     T::IDESC_S);
             };
             // O_t += P_t V: M = 128, N = 64 dims, K = 64 keys; P from TMEM
             // (16 keys per 8 columns), V MN-major.
-            auto mma_pv = [&](int t, uint32_t v_addr, bool accumulate) {
-                const uint64_t dv0 = sdesc_sw128(v_addr, T::KV_TILE, 1024);
+            auto mma_pv = [&](int t, uint64_t dv0, bool accumulate) {
                 umma_ts(tmem + T::O_COL + 64u * t, tmem + 64u * t, dv0, T::IDESC_PV,
                         accumulate ? 1u : 0u);
 #pragma unroll
@@ -242,60 +245,76 @@ __global__ void __launch_bounds__(256, 2)
                     umma_ts_c<true>(tmem + T::O_COL + 64u * t, tmem + 64u * t + 8u * k,
                                     sdesc_add(dv0, k * 2048), T::IDESC_PV);
             };
-            auto pv_tile = [&](int t, uint32_t v_addr, bool acc, uint32_t par) -> bool {
-                if (!mbar_wait(&p_ready[t], par, st)) return false;
+            auto pv_tile = [&](int t, uint64_t dv0, bool acc, uint32_t par) -> bool {
+                if (!mbar_wait_s(pready_a + 8u * t, par, st)) return false;
                 tc_fence_after();
-                mma_pv(t, v_addr, acc);
+                mma_pv(t, dv0, acc);
                 return true;
             };
-            auto act0 = [&](int i) { return i >= off0 && i - off0 < n0; };
-            bool ok = mbar_wait(bar_q, 0, st) && mbar_wait(&full[0], 0, st);
+            // Tile 0 takes part in iterations [off0, n1) (off0 + n0 = n1).
+            auto act0 = [&](int i) { return i >= off0; };
+            bool ok = mbar_wait(bar_q, 0, st) && mbar_wait_s(full_a, 0, st);
             if (ok) {
                 tc_fence_after();
                 if (act0(0)) {
-                    mma_s(0, slot_addr(0));
-                    umma_commit(&s_full[0]);
+                    mma_s(0, dk_base);
+                    umma_commit_s(sfull_a);
                 }
-                mma_s(1, slot_addr(0));
-                umma_commit(&s_full[1]);
-                umma_commit(&empty[0]);
+                mma_s(1, dk_base);
+                umma_commit_s(sfull_a + 8u);
+                umma_commit_s(empty_a);
             }
             // Iteration j: PV_0(j-1), S_0(j), PV_1(j-1), S_1(j).  S of a tile
             // overwrites its P only after the PV that reads it (MMAs from
-            // one thread run in order).
+            // one thread run in order).  ks, kp: ring slot and phase parity
+            // of K_j (position 2j); V_{j-1} sits one position before it.
+            uint32_t ks = 2u % T::NSLOT, kp = (2u / T::NSLOT) & 1u;
             for (int j = 1; j < n1 && ok; ++j) {
-                const int ik = 2 * j, iv = 2 * j - 1;  // K of iteration j, V of j-1
-                ok = mbar_wait(&full[ik % T::NSLOT], slot_par(ik), st) &&
-                     mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st);
+                const uint32_t vs = ks ? ks - 1u : T::NSLOT - 1u;
+                const uint32_t vp = ks ? kp : kp ^ 1u;
+                ok = mbar_wait_s(full_a + 8u * ks, kp, st) && mbar_wait_s(full_a + 8u * vs, vp, st);
                 if (!ok) break;
                 tc_fence_after();
+                const uint64_t dk = sdesc_add(dk_base, ks * T::KV_TILE);
+                const uint64_t dv = sdesc_add(dv_base, vs * T::KV_TILE);
                 if (act0(j - 1)) {
-                    const int l0 = j - 1 - off0;
-                    if (!(ok = pv_tile(0, slot_addr(iv), l0 > 0, l0 & 1))) break;
-                    if (l0 == n0 - 1) umma_commit(&o_final[0]);
+                    const int l0 = j - 1 - off0;  // never tile 0's last block (that is j = n1)
+                    if (!(ok = pv_tile(0, dv, l0 > 0, l0 & 1))) break;
                 }
                 if (act0(j)) {
-                    mma_s(0, slot_addr(ik));
-                    umma_commit(&s_full[0]);
+                    mma_s(0, dk);
+                    umma_commit_s(sfull_a);
                 }
-                if (!(ok = pv_tile(1, slot_addr(iv), j - 1 > 0, (j - 1) & 1))) break;
-                umma_commit(&empty[iv % T::NSLOT]);
-                mma_s(1, slot_addr(ik));
-                umma_commit(&s_full[1]);
-                umma_commit(&empty[ik % T::NSLOT]);
+                if (!(ok = pv_tile(1, dv, j - 1 > 0, (j - 1) & 1))) break;
+                umma_commit_s(empty_a + 8u * vs);
+                mma_s(1, dk);
+                umma_commit_s(sfull_a + 8u);
+                umma_commit_s(empty_a + 8u * ks);
+                ks += 2u;
+                if (ks >= T::NSLOT) {
+                    ks -= T::NSLOT;
+                    kp ^= 1u;
+                }
             }
-            if (ok) {
-                const int jl = n1 - 1, iv = 2 * n1 - 1;
-                ok = mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st);
+            if (ok) {  // V of the last block, one position before K_{n1}'s
+                const int jl = n1 - 1;
+                const uint32_t vs = ks ? ks - 1u : T::NSLOT - 1u;
+                const uint32_t vp = ks ? kp : kp ^ 1u;
+                const uint64_t dv = sdesc_add(dv_base, vs * T::KV_TILE);
+                ok = mbar_wait_s(full_a + 8u * vs, vp, st);
                 if (ok && act0(jl)) {
+                    tc_fence_after();
                     const int l0 = jl - off0;
-                    ok = pv_tile(0, slot_addr(iv), l0 > 0, l0 & 1);
-                    if (ok) umma_commit(&o_final[0]);
+                    ok = pv_tile(0, dv, l0 > 0, l0 & 1);
+                    if (ok) umma_commit_s(ofinal_a);
                 }
-                if (ok) ok = pv_tile(1, slot_addr(iv), jl > 0, jl & 1);
                 if (ok) {
-                    umma_commit(&o_final[1]);
-                    umma_commit(&empty[iv % T::NSLOT]);
+                    tc_fence_after();
+                    ok = pv_tile(1, dv, jl > 0, jl & 1);
+                }
+                if (ok) {
+                    umma_commit_s(ofinal_a + 8u);
+                    umma_commit_s(empty_a + 8u * vs);
                 }
             }
             // No MMA may still be running when TMEM is released.
