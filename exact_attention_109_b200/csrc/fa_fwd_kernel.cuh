@@ -90,9 +90,13 @@ struct FwdTraits {
     static constexpr int LOAD_WARP = 9;
     static constexpr int BIAS_WARP = 10;
     // Register split: softmax warpgroups grow, the MMA/TMA warpgroup shrinks.
-    static constexpr uint32_t REG_SOFTMAX = 200;
-    static constexpr uint32_t REG_CONTROL = 104;
-    static constexpr int REG_BUDGET = 128 * (2 * REG_SOFTMAX + REG_CONTROL);
+    // The causal softmax (diagonal masks) keeps 208; the non-causal MMA
+    // thread needs 104 to hold its descriptors and addresses without
+    // spilling.  Both splits total the same 64,512 registers.
+    static __host__ __device__ constexpr uint32_t reg_softmax(bool causal) { return causal ? 208 : 200; }
+    static __host__ __device__ constexpr uint32_t reg_control(bool causal) { return causal ? 88 : 104; }
+    static constexpr int REG_BUDGET = 128 * (2 * 208 + 88);
+    static_assert(2 * 200 + 104 == 2 * 208 + 88, "both splits use the same registers");
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t IDESC_S = QK8 ? idesc_e4m3_f32(128, BN) : idesc_bf16_f32(128, BN, 0, 0);
     static constexpr uint32_t IDESC_PV =
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tmem = *tmem_slot;
     const AbortState st{abort_flag, p.err};
     if (warp >= 8) {
-      setmaxnreg_dec<T::REG_CONTROL>();
+      setmaxnreg_dec<T::reg_control(CAUSAL)>();
       if (warp == T::LOAD_WARP) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
@@ -402,9 +406,14 @@ __global__ void __launch_bounds__(384, 1)
                                     sdesc_sw128(q_base + T::QK_TILE_BYTES, 16, 1024)};
             const uint64_t dk_base = sdesc_sw128(kv_base, 16, 1024);             // K in slot 0
             const uint64_t dv_base = sdesc_sw128(kv_base, T::CHUNK_BYTES, 1024);  // V in slot 0
-            const uint32_t full_a = smem_u32(full), empty_a = smem_u32(empty);
-            const uint32_t sfull_a = smem_u32(s_full), pready_a = smem_u32(p_ready);
-            const uint32_t phalf_a = smem_u32(p_half), ofinal_a = smem_u32(o_final);
+            // Barrier addresses: one register (the barrier block's base) plus
+            // compile-time offsets, so this thread's register budget stays small.
+            const uint32_t bar_a = smem_u32(bars);
+            constexpr uint32_t FULL = 8u * 1, EMPTY = FULL + 8u * T::NSLOT, SFULL = EMPTY + 8u * T::NSLOT;
+            constexpr uint32_t PREADY = SFULL + 16u, OFINAL = PREADY + 16u;
+            constexpr uint32_t PHALF = OFINAL + 16u + 8u + 32u;  // after mma_done, bias_full/empty
+            const uint32_t full_a = bar_a + FULL, empty_a = bar_a + EMPTY, sfull_a = bar_a + SFULL;
+            const uint32_t pready_a = bar_a + PREADY, phalf_a = bar_a + PHALF, ofinal_a = bar_a + OFINAL;
             // S_t = Q_t K^T : M=128, N=128, K=D, both operands K-major;
             // each MMA consumes 32 bytes of every row (16 bf16 or 32 e4m3).
             // dk: the descriptor of the K slot; K steps add byte offsets.
@@ -528,7 +537,7 @@ __global__ void __launch_bounds__(384, 1)
       }
     } else {
         // ------------------------------------------------ softmax warpgroups
-        setmaxnreg_inc<T::REG_SOFTMAX>();
+        setmaxnreg_inc<T::reg_softmax(CAUSAL)>();
         const int t = warp >> 2;         // query tile
         const int lg = warp & 3;         // TMEM lane group of this warp
         const int r = lg * 32 + lane;    // row within the tile = TMEM lane
