@@ -192,17 +192,24 @@ __global__ void __launch_bounds__(256, 2)
         __syncwarp();
       } else if (warp == T::MMA_WARP) {
         // ------------------------------------------------ MMA issuer
+        // This thread's instruction stream is on the kernel's critical path:
+        // descriptors and barrier addresses are built once, and the ring
+        // position is an unsigned counter (a mask and a shift per use).
         if (lane == 0) {
             const uint32_t q_base = smem_u32(smem + T::Q_OFF);
             const uint32_t kv_base = smem_u32(smem + T::KV_OFF);
-            auto slot_addr = [&](int idx) {
-                return kv_base + static_cast<uint32_t>((idx % T::NSLOT) * T::TILE_BYTES);
-            };
-            auto slot_par = [&](int idx) { return static_cast<uint32_t>((idx / T::NSLOT) & 1); };
             const uint64_t dq0 = sdesc_sw128(q_base, 16, 1024);
-            // S = Q K^T: M=128, N=128, K=D, both K-major.
-            auto mma_s = [&](uint32_t k_addr) {
-                const uint64_t dk0 = sdesc_sw128(k_addr, 16, 1024);
+            const uint64_t dk_base = sdesc_sw128(kv_base, 16, 1024);             // K in slot 0
+            const uint64_t dv_base = sdesc_sw128(kv_base, T::CHUNK_BYTES, 1024);  // V in slot 0
+            const uint32_t qfull_a = smem_u32(q_full), qempty_a = smem_u32(q_empty);
+            const uint32_t full_a = smem_u32(full), empty_a = smem_u32(empty);
+            const uint32_t sfull_a = smem_u32(s_full), pready_a = smem_u32(p_ready);
+            const uint32_t phalf_a = smem_u32(p_half), ofinal_a = smem_u32(o_final);
+            const uint32_t ofree_a = smem_u32(o_free);
+            auto slot = [](uint32_t idx) { return idx % static_cast<uint32_t>(T::NSLOT); };
+            auto slot_par = [](uint32_t idx) { return (idx / static_cast<uint32_t>(T::NSLOT)) & 1u; };
+            // S = Q K^T: M=128, N=128, K=D, both K-major; dk: the K slot.
+            auto mma_s = [&](uint64_t dk0) {
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k) {
                     const uint32_t off = (k >> 2) * T::CHUNK_BYTES + (k & 3) * 32;
@@ -213,8 +220,7 @@ __global__ void __launch_bounds__(256, 2)
                 }
             };
             // O += P V: M=128, N=D, K=128 keys; P from TMEM, V MN-major.
-            auto mma_pv = [&](uint32_t v_addr, bool accumulate, int k0, int k1) {
-                const uint64_t dv0 = sdesc_sw128(v_addr, T::CHUNK_BYTES, 1024);
+            auto mma_pv = [&](uint64_t dv0, bool accumulate, int k0, int k1) {
 #pragma unroll
                 for (int k = k0; k < k1; ++k) {
                     if (k == 0)
@@ -224,10 +230,12 @@ __global__ void __launch_bounds__(256, 2)
                                         T::IDESC_PV);
                 }
             };
+            auto kdesc = [&](uint32_t idx) { return sdesc_add(dk_base, slot(idx) * T::TILE_BYTES); };
+            auto vdesc = [&](uint32_t idx) { return sdesc_add(dv_base, slot(idx) * T::TILE_BYTES); };
             bool ok = true;
-            int idx = 0;  // K/V tiles consumed so far
-            int jb = 0;   // key blocks done so far (s_full / p_ready phases)
-            int ni = 0;   // tiles done so far (q_full / o_final / o_free phases)
+            uint32_t idx = 0;  // K/V tiles consumed so far
+            uint32_t jb = 0;   // key blocks done so far (s_full / p_ready phases)
+            uint32_t ni = 0;   // tiles done so far (q_full / o_final / o_free phases)
             for (int it = blockIdx.x; it < items && ok; it += gridDim.x) {
                 int qt, bh;
                 decode(it, qt, bh);
@@ -235,51 +243,52 @@ __global__ void __launch_bounds__(256, 2)
                 // S of the tile's first block overwrites the previous tile's
                 // last P only after the PV that read it (MMAs from one thread
                 // run in order).
-                if (!(ok = mbar_wait(q_full, ni & 1, st) &&
-                           mbar_wait(&full[idx % T::NSLOT], slot_par(idx), st)))
+                if (!(ok = mbar_wait_s(qfull_a, ni & 1u, st) &&
+                           mbar_wait_s(full_a + 8u * slot(idx), slot_par(idx), st)))
                     break;
                 tc_fence_after();
-                mma_s(slot_addr(idx));
-                umma_commit(s_full);
-                umma_commit(&empty[idx % T::NSLOT]);
+                mma_s(kdesc(idx));
+                umma_commit_s(sfull_a);
+                umma_commit_s(empty_a + 8u * slot(idx));
                 ++idx;
-                if (n == 1) umma_commit(q_empty);
+                if (n == 1) umma_commit_s(qempty_a);
                 for (int i = 0; i < n && ok; ++i, ++jb) {
-                    const int iv = idx;  // V of block i
-                    const uint32_t par = jb & 1;
-                    if (!(ok = mbar_wait(&full[iv % T::NSLOT], slot_par(iv), st))) break;
+                    const uint32_t iv = idx;  // V of block i
+                    const uint32_t par = jb & 1u;
+                    if (!(ok = mbar_wait_s(full_a + 8u * slot(iv), slot_par(iv), st))) break;
                     // the first PV of a tile overwrites O: the softmax warps
                     // must have read the previous tile's O out of TMEM
-                    if (i == 0 && ni > 0 && !(ok = mbar_wait(o_free, (ni - 1) & 1, st))) break;
+                    if (i == 0 && ni > 0 && !(ok = mbar_wait_s(ofree_a, (ni - 1) & 1u, st))) break;
+                    const uint64_t dv = vdesc(iv);
                     if constexpr (T::PSPLIT) {
-                        if (!(ok = mbar_wait(p_half, par, st))) break;
+                        if (!(ok = mbar_wait_s(phalf_a, par, st))) break;
                         tc_fence_after();
-                        mma_pv(slot_addr(iv), i > 0, 0, T::BN / 32);
-                        if (!(ok = mbar_wait(p_ready, par, st))) break;
+                        mma_pv(dv, i > 0, 0, T::BN / 32);
+                        if (!(ok = mbar_wait_s(pready_a, par, st))) break;
                         tc_fence_after();
-                        mma_pv(slot_addr(iv), true, T::BN / 32, T::BN / 16);
+                        mma_pv(dv, true, T::BN / 32, T::BN / 16);
                     } else {
-                        if (!(ok = mbar_wait(p_ready, par, st))) break;
+                        if (!(ok = mbar_wait_s(pready_a, par, st))) break;
                         tc_fence_after();
-                        mma_pv(slot_addr(iv), i > 0, 0, T::BN / 16);
+                        mma_pv(dv, i > 0, 0, T::BN / 16);
                     }
-                    umma_commit(&empty[iv % T::NSLOT]);
+                    umma_commit_s(empty_a + 8u * slot(iv));
                     ++idx;
                     if (i + 1 < n) {
                         // S of the next block overwrites P after this PV has
                         // read it; its completion also covers this PV, so the
                         // softmax may then rescale O.
-                        if (!(ok = mbar_wait(&full[idx % T::NSLOT], slot_par(idx), st))) break;
+                        if (!(ok = mbar_wait_s(full_a + 8u * slot(idx), slot_par(idx), st))) break;
                         tc_fence_after();
-                        mma_s(slot_addr(idx));
-                        umma_commit(s_full);
-                        umma_commit(&empty[idx % T::NSLOT]);
+                        mma_s(kdesc(idx));
+                        umma_commit_s(sfull_a);
+                        umma_commit_s(empty_a + 8u * slot(idx));
                         ++idx;
-                        if (i + 2 == n) umma_commit(q_empty);  // the tile's last S
+                        if (i + 2 == n) umma_commit_s(qempty_a);  // the tile's last S
                     }
                 }
                 if (!ok) break;
-                umma_commit(o_final);
+                umma_commit_s(ofinal_a);
                 ++ni;
             }
             umma_commit(mma_done);
